@@ -1,0 +1,369 @@
+"""Benchmark of one absorbed-MLA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3] [--impl ours|reference]
+
+A step is the whole hot path for one layer: mla_append_latent (this step's
+cache rows), mla_absorb_q and mla_decode_attn (split-KV attention, LSE
+combine, W_UV) over a batch of synthetic sequences whose latent cache is
+resident in HBM.  The default workload is DeepSeek-V3-shaped decode: 16
+sequences, 128 heads, context 32768, 64-token pages, shuffled page table.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronise, timed with CUDA events on the launching stream; the
+latent cache (604 MB at the default workload) is larger than L2, so no L2
+flush is inserted.  Multi-GPU (torchrun): every rank runs its own replica on
+its own batch (data parallel over sequences, no collective on the data path)
+and the slowest rank's time is reported.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (float64 numpy, absorbed form) on a
+bounded sample of the same workload on the host cores, as the comparison arm.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workload as W  # noqa: E402
+
+METRIC = "MLA latent decode tokens/s; HBM GB/s and TFLOPS as fraction of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def describe(w: W.Workload) -> dict:
+    d = {"workload": f"{w.name}: batch {w.batch}, {w.nq} query token(s)/seq, {w.n_heads} heads, "
+                     + (f"context {w.context}" if w.context else f"context U[{w.ragged[0]},{w.ragged[1]}]")
+                     + f", d_c {w.d_c}, d_rope {w.d_rope}, page {w.page_size}",
+         "batch": w.batch, "nq": w.nq, "n_heads": w.n_heads, "d_c": w.d_c, "d_rope": w.d_rope,
+         "qk_nope": w.qk_nope, "v_head": w.v_head, "d_model": w.d_model, "page_size": w.page_size,
+         "context": w.context if w.context else list(w.ragged), "page_table": "shuffled",
+         "l2": "inputs larger than L2: the latent cache streamed each step exceeds the 126 MB L2"}
+    return d
+
+
+def algorithmic_counts(w: W.Workload, lens: np.ndarray) -> dict:
+    """Bytes and flops mla_decode_attn must move / compute (cache read once per
+    sequence, W_UV once, q_lat in, out written), per launch."""
+    R = w.row
+    T = w.tokens
+    cache = int(lens.sum()) * R * 2
+    nbytes = cache + w.n_heads * w.v_head * w.d_c * 2 + T * w.n_heads * R * 2 + T * w.n_heads * w.v_head * 2
+    # visible keys per query token: N_b - nq + 1 + i
+    keys = sum(int(n) - w.nq + 1 + i for n in lens for i in range(w.nq))
+    flops = keys * w.n_heads * 2 * (R + w.d_c) + T * w.n_heads * 2 * w.d_c * w.v_head
+    return {"bytes": nbytes, "flops": flops, "cache_bytes": cache}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import head_latent_attention_07_b200 as M
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    x = W.make_decode_inputs(w, seed=args.seed + rank)
+    to_bf16 = lambda b: torch.from_numpy(np.ascontiguousarray(b)).view(torch.bfloat16).to(dev)
+    to_i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    dims = M.MlaDims(n_heads=w.n_heads, d_c=w.d_c, d_rope=w.d_rope, qk_nope=w.qk_nope, v_head=w.v_head,
+                     d_model=w.d_model, page_size=w.page_size)
+    T = w.tokens
+    h, q = to_bf16(x.bits["h"]), to_bf16(x.bits["q"])
+    w_dkv, w_uk, w_uv = to_bf16(x.bits["w_dkv"]), to_bf16(x.bits["w_uk"]), to_bf16(x.bits["w_uv"])
+    pool = to_bf16(x.bits["pool"])
+    del x.bits["pool"]
+    page_table = to_i32(x.page_table)
+    seq_lens, seq_idx, pos = to_i32(x.lens), to_i32(x.h_seq_idx), to_i32(x.pos)
+    q_lat = torch.empty((w.batch, w.nq, w.n_heads, w.row), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((w.batch, w.nq, w.n_heads, w.v_head), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.nq, w.n_heads), dtype=torch.float32, device=dev)
+    ws = torch.empty(M.mla_decode_workspace_bytes(dims, w.batch, w.nq), dtype=torch.uint8, device=dev)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev_pairs = []
+
+    def step(h_, q_, seq_idx_, pos_, seq_lens_, record=False):
+        M.mla_append_latent(dims, h_, w_dkv, seq_idx_, pos_, page_table, pool, dev_status=status, stream=stream)
+        M.mla_absorb_q(dims, q_, pos_, w_uk, q_lat.view(T, w.n_heads, w.row), stream=stream)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        M.mla_decode_attn(dims, q_lat, pool, page_table, seq_lens_, w_uv, ws, out, lse, dev_status=status,
+                          stream=stream)
+        if record:
+            e1.record(stream)
+            ev_pairs.append((e0, e1))
+
+    launches_per_step = 4  # append, absorb, decode split, decode combine
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        step(h, q, seq_idx, pos, seq_lens)
+    barrier()
+    assert M.mla_status_read(status, stream) == 0, "device status after warm-up"
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    sampler.start()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(h, q, seq_idx, pos, seq_lens, record=True)
+    t1.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    ms_total = t0.elapsed_time(t1)
+    decode_ms = [a.elapsed_time(b) for a, b in ev_pairs]
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    host = {k: v.cpu().pin_memory() for k, v in (("h", h), ("q", q), ("seq_idx", seq_idx), ("pos", pos),
+                                                  ("seq_lens", seq_lens))}
+    dbuf = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k in host:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        step(dbuf["h"], dbuf["q"], dbuf["seq_idx"], dbuf["pos"], dbuf["seq_lens"])
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    assert M.mla_status_read(status, stream) == 0, "device status after timing"
+
+    times = torch.tensor([ms_total, e2e_ms, float(np.mean(decode_ms))], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms, dec_ms = times.tolist()
+    return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": dec_ms, "clocks": clocks,
+            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+class OracleArm:
+    """The CPU oracle's absorbed form (float64 numpy), as it stands, on query
+    tokens of this workload.  Inputs are drawn once; each measure() call runs
+    whole query tokens (all heads) until ~budget_s of host time is spent."""
+
+    def __init__(self, w: W.Workload, seed: int):
+        from oracle import mla as O
+        self.O, self.w = O, w
+        try:
+            from threadpoolctl import threadpool_info
+            self.cores = max((int(i.get("num_threads", 1)) for i in threadpool_info()), default=1)
+        except Exception:  # noqa: BLE001
+            self.cores = 1
+        # a uniform workload: one sequence's cache stands for all (same work per query token)
+        x = W.make_decode_inputs(dataclasses.replace(w, batch=1) if w.context else w, seed=seed)
+        self.args = dict(h=x.f64("h"), h_seq_idx=x.h_seq_idx, h_pos=x.h_pos, q=x.f64("q"), q_pos=x.pos,
+                         pool=_Widen(x.bits["pool"]), page_table=x.page_table, lens=x.lens,
+                         nq=x.workload.nq, w_dkv=x.f64("w_dkv"), w_uk=x.f64("w_uk"), w_uv=x.f64("w_uv"),
+                         d_c=w.d_c)
+        self.tokens = x.workload.tokens
+        self.done = 0
+
+    def measure(self, budget_s: float):
+        n, t0 = 0, time.perf_counter()
+        while n == 0 or time.perf_counter() - t0 < budget_s:
+            self.O.decode_step(**self.args, form="absorbed", queries=[self.done % self.tokens])
+            self.done += 1
+            n += 1
+        el = time.perf_counter() - t0
+        ctx = f"context {self.w.context}" if self.w.context else "ragged contexts"
+        return n / el, (f"oracle absorbed form (float64 numpy): {n} query token(s) x {self.w.n_heads} heads "
+                        f"over {ctx} in {el:.1f} s, scaled to tokens/s")
+
+
+class _Widen:
+    """bf16 pool bits read as float32 rows on demand."""
+
+    def __init__(self, bits):
+        self.b, self.shape = bits, bits.shape
+
+    def __getitem__(self, i):
+        return W.bf16_to_f32(self.b[i])
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="v3", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    w = W.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        # each step: the oracle on a bounded sample (one query token at least)
+        arm = OracleArm(w, args.seed)
+        per_step = []
+        budget = max(0.2, min(8.0, 120.0 / (args.steps + args.warmup)))
+        for i in range(args.warmup + args.steps):
+            v, sample = arm.measure(budget)
+            if i >= args.warmup:
+                per_step.append(v)
+        value = float(np.mean(per_step))
+        cores = arm.cores
+        ms = 1000.0 * w.tokens / value
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": describe(w),
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    r = run_ours(args, w, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, src = load_peaks()
+    cnt = algorithmic_counts(w, r["lens"])
+    T = w.tokens
+    value = world * T * args.steps / (r["ms_total"] / 1000.0)
+    dec_s = r["decode_ms"] / 1000.0
+    gbs = cnt["bytes"] / dec_s / 1e9
+    tfs = cnt["flops"] / dec_s / 1e12
+    t_hbm = cnt["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = cnt["flops"] / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    roof = ({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s"} if bound == "hbm" else
+            {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"})
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "mla_decode_attn (split + combine launches)"
+    roof["peak_source"] = f"{src} (MEASURED_PEAKS.json burst figures)" if src == "measured" else "fallback"
+    roof["hbm_frac"] = gbs / peaks["hbm_gbs"]
+    roof["tensor_frac"] = tfs / peaks["bf16_tflops"]
+    roof["time_us"] = r["decode_ms"] * 1000.0
+    roof["bytes_per_launch"] = cnt["bytes"]
+    roof["flops_per_launch"] = cnt["flops"]
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_total"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**describe(w), "parallelism": f"dp{world} (independent replicas)"},
+            "roofline": roof,
+            "e2e": {"value": world * T * args.steps / (r["e2e_ms"] / 1000.0), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "gpu_launches": r["launches"], "clocks": r["clocks"]}
+    if world == 1 and not args.no_cpu_baseline:
+        arm = OracleArm(w, args.seed)
+        v, sample = arm.measure(args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": arm.cores, "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+// C ABI of libmla_b200.so: argument validation, workspace sizing, launches.
+// The declarations and the contract of every entry point are in include/mla.h.
+#include <math.h>
+
+#include "../../include/mla.h"
+#include "decode.h"
+#include "plan.cuh"
+
+namespace {
+
+constexpr float kDefaultTheta = 10000.f;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by all calls.  d_rope == 0 is refused: without the
+// decoupled RoPE channels W_UK cannot be folded into the query (the rotation
+// sits between W_Q and W_UK), so an "absorbed" result would be wrong.
+int check_dims(const mla_dims* d) {
+  if (d == nullptr) return MLA_ERR_INVALID_ARG;
+  if (d->n_heads < 1 || d->d_c < 1 || d->qk_nope < 1 || d->v_head < 1 || d->d_model < 1 ||
+      d->page_size < 1 || d->d_rope < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (d->d_rope == 0) return MLA_ERR_UNSUPPORTED;
+  if (d->n_heads > 128 || d->d_c > 512 || d->d_c % 8 || d->d_rope % 8 || d->d_rope > 256 ||
+      d->qk_nope % 8 || d->qk_nope > 1024 || d->v_head % 8 || d->v_head > 1024 ||
+      d->d_model % 8 || d->page_size > 256)
+    return MLA_ERR_UNSUPPORTED;
+  // one cache page and the query rows of a CTA must fit in shared memory
+  if (mla::decode_simt_smem_bytes(d->d_c, d->d_rope, d->page_size) > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+  if (!(d->softmax_scale >= 0.f) || isinf(d->softmax_scale) || !(d->rope_theta >= 0.f) ||
+      isinf(d->rope_theta))
+    return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+float eff_scale(const mla_dims* d) {
+  return d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)(d->qk_nope + d->d_rope));
+}
+float eff_theta(const mla_dims* d) { return d->rope_theta > 0.f ? d->rope_theta : kDefaultTheta; }
+
+int device_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t part_o_bytes, part_lse_bytes, total;
+};
+
+// Workspace for at most (#SMs + batch) split pieces of nq*H rows each.
+WsLayout ws_layout(const mla_dims* d, int batch, int nq, int sms) {
+  const size_t pieces = (size_t)mla::max_pieces(sms, batch);
+  const size_t rows = (size_t)nq * d->n_heads;
+  WsLayout w;
+  w.part_o_bytes = align256(pieces * rows * d->d_c * sizeof(float));
+  w.part_lse_bytes = align256(pieces * rows * sizeof(float));
+  w.total = w.part_o_bytes + w.part_lse_bytes;
+  return w;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int mla_append_latent(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv,
+                      const int32_t* seq_idx, const int32_t* pos, const int32_t* page_table,
+                      int32_t batch, int32_t max_pages, mla_bf16* pool, int32_t num_pages,
+                      int32_t n_tokens, int32_t* dev_status, void* stream) {
+  int st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (n_tokens < 0 || batch < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!h || !w_dkv || !seq_idx || !pos || !page_table || !pool) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(seq_idx) || !aligned16(pos) ||
+      !aligned16(page_table) || !aligned16(pool) || (dev_status && !aligned16(dev_status)))
+    return MLA_ERR_MISALIGNED;
+  if ((int64_t)max_pages * dims->page_size > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+  mla::AppendArgs a;
+  a.h = h; a.w_dkv = w_dkv; a.seq_idx = seq_idx; a.pos = pos; a.page_table = page_table;
+  a.pool = pool; a.dev_status = dev_status; a.n_tokens = n_tokens; a.d_model = dims->d_model;
+  a.d_c = dims->d_c; a.d_rope = dims->d_rope; a.page_size = dims->page_size; a.batch = batch;
+  a.max_pages = max_pages; a.num_pages = num_pages; a.theta = eff_theta(dims);
+  return cuda_status(mla::launch_append_latent(a, (cudaStream_t)stream));
+}
+
+int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
+                 const mla_bf16* w_uk, mla_bf16* q_lat, int32_t n_tokens, void* stream) {
+  int st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (n_tokens < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!q || !pos || !w_uk || !q_lat) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(pos) || !aligned16(w_uk) || !aligned16(q_lat)) return MLA_ERR_MISALIGNED;
+  mla::AbsorbArgs a;
+  a.q = q; a.pos = pos; a.w_uk = w_uk; a.q_lat = q_lat; a.n_tokens = n_tokens;
+  a.n_heads = dims->n_heads; a.qk_nope = dims->qk_nope; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
+  a.theta = eff_theta(dims);
+  return cuda_status(mla::launch_absorb_q(a, (cudaStream_t)stream));
+}
+
+size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t nq) {
+  if (check_dims(dims) != MLA_OK || batch < 1 || batch > mla::kMaxBatch || nq < 1 || nq > 16) return 0;
+  int sms = 0;
+  if (device_sms(&sms) != MLA_OK) return 0;
+  return ws_layout(dims, batch, nq, sms).total;
+}
+
+int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
+                    const int32_t* page_table, const int32_t* seq_lens, int32_t batch,
+                    int32_t nq, int32_t max_pages, int32_t num_pages, const mla_bf16* w_uv,
+                    void* workspace, size_t ws_bytes, mla_bf16* out, float* lse,
+                    int32_t* dev_status, void* stream) {
+  int st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (batch < 1 || nq < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (batch > mla::kMaxBatch || nq > 16) return MLA_ERR_UNSUPPORTED;
+  if ((int64_t)max_pages * dims->page_size > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+  if (!q_lat || !pool || !page_table || !seq_lens || !w_uv || !workspace || !out) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_lat) || !aligned16(pool) || !aligned16(page_table) || !aligned16(seq_lens) ||
+      !aligned16(w_uv) || !aligned16(workspace) || !aligned16(out) || (lse && !aligned16(lse)) ||
+      (dev_status && !aligned16(dev_status)))
+    return MLA_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_sms(&sms)) != MLA_OK) return st;
+  const WsLayout wl = ws_layout(dims, batch, nq, sms);
+  if (ws_bytes < wl.total) return MLA_ERR_WORKSPACE;
+
+  mla::DecodeArgs a;
+  a.q_lat = q_lat; a.pool = pool; a.page_table = page_table; a.seq_lens = seq_lens; a.w_uv = w_uv;
+  a.out = out; a.lse = lse; a.dev_status = dev_status;
+  a.part_o = reinterpret_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + wl.part_o_bytes);
+  a.batch = batch; a.nq = nq; a.n_heads = dims->n_heads; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
+  a.v_head = dims->v_head; a.page_size = dims->page_size; a.max_pages = max_pages;
+  a.num_pages = num_pages; a.scale = eff_scale(dims);
+  const int groups = mla::decode_simt_row_groups(nq * dims->n_heads);
+  int G = (2 * sms + groups - 1) / groups;
+  a.G = G < 1 ? 1 : (G > sms ? sms : G);
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
+  return cuda_status(mla::launch_decode_combine(a, s));
+}
+
+int mla_status_read(const int32_t* dev_status, void* stream) {
+  if (dev_status == nullptr) return MLA_ERR_INVALID_ARG;
+  int32_t v = 0;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpy(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  return v;
+}
+
+int mla_status_clear(int32_t* dev_status, void* stream) {
+  if (dev_status == nullptr) return MLA_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), (cudaStream_t)stream));
+}
+
+const char* mla_status_string(int status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: null pointer, bad size or count";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: dimensions not implemented by this build";
+    case MLA_ERR_MISALIGNED: return "MLA_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace too small";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: CUDA runtime error";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a bounded device wait ran out";
+    case MLA_ERR_RANGE: return "MLA_ERR_RANGE: page id, position or length out of range";
+    default: return "unknown mla_status";
+  }
+}
+
+const char* mla_version(void) { return "mla_b200 0.1.0 sm_100a"; }
+
+}  // extern "C"

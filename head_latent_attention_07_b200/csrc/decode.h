@@ -1,0 +1,54 @@
+// Internal interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mla {
+
+struct DecodeArgs {
+  const uint16_t* q_lat;      // [B, nq, H, R]
+  const uint16_t* pool;       // [num_pages, P, R]
+  const int32_t* page_table;  // [B, max_pages]
+  const int32_t* seq_lens;    // [B]
+  const uint16_t* w_uv;       // [H, d_v, d_c]
+  uint16_t* out;              // [B, nq, H, d_v]
+  float* lse;                 // [B, nq, H] or null
+  float* part_o;              // [pieces, nq*H, d_c]
+  float* part_lse;            // [pieces, nq*H]
+  int32_t* dev_status;        // or null
+  int batch, nq, n_heads, d_c, d_rope, v_head, page_size, max_pages, num_pages;
+  int G;                      // split workers
+  float scale;
+};
+
+struct AppendArgs {
+  const uint16_t* h;          // [T, D]
+  const uint16_t* w_dkv;      // [R, D]
+  const int32_t* seq_idx;     // [T]
+  const int32_t* pos;         // [T]
+  const int32_t* page_table;  // [B, max_pages]
+  uint16_t* pool;             // [num_pages, P, R]
+  int32_t* dev_status;
+  int n_tokens, d_model, d_c, d_rope, page_size, batch, max_pages, num_pages;
+  float theta;
+};
+
+struct AbsorbArgs {
+  const uint16_t* q;          // [T, H, d_n + d_r]
+  const int32_t* pos;         // [T]
+  const uint16_t* w_uk;       // [H, d_n, d_c]
+  uint16_t* q_lat;            // [T, H, d_c + d_r]
+  int n_tokens, n_heads, qk_nope, d_c, d_rope;
+  float theta;
+};
+
+size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);
+int decode_simt_row_groups(int rows_total);
+cudaError_t launch_decode_split_simt(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream);
+cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
+
+}  // namespace mla

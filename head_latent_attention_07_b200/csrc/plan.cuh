@@ -1,0 +1,126 @@
+// Split-KV schedule shared by the decode split kernels and the combine kernel.
+//
+// The pages of all sequences are laid end to end (sequence 0's pages, then
+// sequence 1's, ...).  That flat list is cut into contiguous chunks of `chunk`
+// pages; worker w processes flat pages [w*chunk, (w+1)*chunk).  A worker's chunk
+// may end inside one sequence and continue into the next.  Each overlap of a
+// worker with a sequence is a "piece"; a piece writes one partial result
+// (softmax-normalised latent output and log-sum-exp per row) to the workspace.
+// The pieces of sequence b are consecutive: piece_begin[b] .. piece_begin[b] +
+// npieces[b] - 1, worker w's piece of b being piece_begin[b] + (w - w_first[b]).
+// With chunk >= ceil(total / G) at most G workers are busy, so there are at
+// most G + batch - 1 pieces.
+//
+// Every CTA rebuilds this schedule from seq_lens in shared memory (two block
+// scans over the batch), so no planning launch and no metadata buffer exist.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+constexpr int kMaxBatch = 1024;   // sequences per decode call
+constexpr int kMinChunk = 4;      // pages: keeps per-piece overhead bounded
+
+struct PlanSmem {
+  int start[kMaxBatch + 1];        // first flat page of each sequence; start[B] = total
+  int piece_begin[kMaxBatch + 1];  // first piece of each sequence; piece_begin[B] = #pieces
+  int chunk;                       // pages per worker
+  int warp_tot[32];
+};
+
+// Host-side bound on the number of pieces, used for workspace sizing.
+inline int64_t max_pieces(int G, int batch) { return (int64_t)G + batch; }
+
+// Number of pages of sequence b; 0 (and a recorded range error) when its
+// length is outside [nq, max_pages * page_size].
+__device__ __forceinline__ int seq_pages(const int32_t* seq_lens, int b, int nq, int max_pages,
+                                         int page_size, int32_t* dev_status) {
+  int len = seq_lens[b];
+  if (len < nq || len > max_pages * page_size) {
+    record_status(dev_status, MLA_ERR_RANGE);
+    return 0;
+  }
+  return (len + page_size - 1) / page_size;
+}
+
+// Block-wide exclusive scan of one int per thread; returns the exclusive prefix
+// and writes the block total to *total.  All threads of the block must call it.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = (blockDim.x + 31) >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nwarps ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    warp_tot[lane] = t;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  int excl = x - v + (warp > 0 ? warp_tot[warp - 1] : 0);
+  *total = warp_tot[nwarps - 1];
+  __syncthreads();
+  return excl;
+}
+
+// Fills ps->start, ps->piece_begin and ps->chunk for `batch` sequences and G workers.
+__device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens, int batch, int nq, int max_pages,
+                           int page_size, int G, int32_t* dev_status) {
+  // pass 1: pages per sequence -> start offsets
+  int carry = 0;
+  for (int base = 0; base < batch; base += blockDim.x) {
+    int b = base + threadIdx.x;
+    int v = b < batch ? seq_pages(seq_lens, b, nq, max_pages, page_size,
+                                  blockIdx.x == 0 && blockIdx.y == 0 ? dev_status : nullptr)
+                      : 0;
+    int tot;
+    int ex = block_exclusive_scan(v, ps->warp_tot, &tot);
+    if (b < batch) ps->start[b] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) {
+    ps->start[batch] = carry;
+    int c = (carry + G - 1) / G;
+    ps->chunk = c < kMinChunk ? kMinChunk : c;
+  }
+  __syncthreads();
+  const int chunk = ps->chunk;
+  // pass 2: pieces per sequence -> piece_begin
+  carry = 0;
+  for (int base = 0; base < batch; base += blockDim.x) {
+    int b = base + threadIdx.x;
+    int v = 0;
+    if (b < batch) {
+      int s = ps->start[b], e = ps->start[b + 1];
+      v = e > s ? (e - 1) / chunk - s / chunk + 1 : 0;
+    }
+    int tot;
+    int ex = block_exclusive_scan(v, ps->warp_tot, &tot);
+    if (b < batch) ps->piece_begin[b] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) ps->piece_begin[batch] = carry;
+  __syncthreads();
+}
+
+// Sequence containing flat page f (start[b] <= f < start[b+1]); f < total.
+__device__ __forceinline__ int seq_of_flat_page(const PlanSmem* ps, int batch, int f) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (ps->start[mid] <= f) lo = mid; else hi = mid - 1;
+  }
+  return lo;  // the largest such b, so empty sequences sharing its start are skipped
+}
+
+}  // namespace mla

@@ -1,0 +1,188 @@
+/*
+ * mla.h - C ABI of the B200 (sm_100a) absorbed Multi-Head Latent Attention
+ * decode library (libmla_b200.so).
+ *
+ * One decode step of one attention layer is three calls, in this order:
+ *   mla_append_latent  write this step's latent-cache rows [c_t || k_t^R]
+ *   mla_absorb_q       fold W_UK into the queries, rotate their RoPE part
+ *   mla_decode_attn    split-KV attention over the paged latent cache,
+ *                      log-sum-exp combine of the splits, then W_UV
+ * Keys and values are never decompressed: every cached token holds only its
+ * latent c_t (d_c scalars) and its decoupled RoPE key k_t^R (d_rope scalars).
+ *
+ * Sources (page title, section):
+ *   [eyestech-pypi]  "eyestech-mla 1.0.0" package description: "Key Architectural
+ *                    Highlights" (576 = 512 + 64 scalars per token; query
+ *                    absorption), quickstart "Autoregressive MLA Decoding with
+ *                    Query Absorption" (decode step appends to the cache, 1024 -> 1025).
+ *   [eyestech-blog]  "DeepSeek MLA Architecture: How It Cuts KV Cache by 93%",
+ *                    sec. 2 "Query Matrix Absorption" (q~ = W_UK^T q).
+ *   [from-scratch]   "mla-from-scratch" README, "Absorption, and why RoPE breaks it"
+ *                    (content + positional score; W_UV applied once after attending
+ *                    over latents; refuse to build without decoupled RoPE).
+ *   [distaisys]      "Deep-Dive: Multi-Head Latent Attention (MLA) and Low-Rank KV
+ *                    Cache Compression in DeepSeek-V3", sec. 2 (c = W_DKV h,
+ *                    k = W_UK c, v = W_UV c) and sec. 3 (weight layouts, softmax).
+ *   [songhuiming]    "MHA vs MLA KV cache comparison", "MLA ... Step-by-step for
+ *                    t100" (append the new latent, then attend over all of them).
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense, row-major (last index fastest), on the current CUDA
+ *     device unless stated.  "bf16" buffers hold IEEE bfloat16 bit patterns.
+ *   - Every device pointer must be 16-byte aligned (MLA_ERR_MISALIGNED).
+ *   - The caller owns every buffer.  The library allocates no device or host
+ *     memory and keeps no state between calls; calls are asynchronous on
+ *     `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *   - Host-checkable errors return a negative mla_status before anything is
+ *     launched.  Errors only the device can see (a page id outside the pool, a
+ *     sequence length outside the page table, a bounded wait that ran out) are
+ *     recorded, first one wins, in the caller's int32 status word `dev_status`
+ *     (may be NULL) and the offending access is skipped: no kernel traps.
+ *   - RoPE: channel pair (2i, 2i+1) rotates by pos * theta^(-2i/d_rope), the
+ *     angle evaluated in double precision; pos = cache index of the token.
+ *   - bf16 outputs are rounded to nearest even from fp32 accumulators.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t mla_bf16; /* bfloat16 bit pattern */
+
+/* Layer dimensions.  Names follow the pages: d_c = kv_lora_rank (latent width),
+ * d_rope = decoupled RoPE width (qk_rope_dim), qk_nope = per-head non-rotary
+ * query/key width d_h, v_head = per-head value width, d_model = D. */
+typedef struct mla_dims {
+  int32_t n_heads;      /* H, 1..128 */
+  int32_t d_c;          /* multiple of 8 */
+  int32_t d_rope;       /* even, multiple of 8, > 0: absorption needs decoupled RoPE */
+  int32_t qk_nope;      /* multiple of 8 */
+  int32_t v_head;       /* multiple of 8 */
+  int32_t d_model;      /* multiple of 8 */
+  int32_t page_size;    /* tokens per latent-cache page: 64 */
+  float softmax_scale;  /* 0 selects 1/sqrt(qk_nope + d_rope) */
+  float rope_theta;     /* 0 selects 10000 */
+} mla_dims;
+
+typedef enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,  /* NULL pointer, non-positive size, bad count */
+  MLA_ERR_UNSUPPORTED = -2,  /* dimensions this build does not implement */
+  MLA_ERR_MISALIGNED = -3,   /* a pointer is not 16-byte aligned */
+  MLA_ERR_WORKSPACE = -4,    /* workspace smaller than mla_decode_workspace_bytes */
+  MLA_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed */
+  MLA_ERR_TIMEOUT = -6,      /* device: a bounded wait inside a kernel ran out */
+  MLA_ERR_RANGE = -7         /* device: page id / position / length out of range */
+} mla_status;
+
+/*
+ * mla_append_latent - write this step's latent-cache rows.
+ *
+ * For each token t (0 <= t < n_tokens) with hidden state h[t] (length d_model):
+ *   [c_t || k^_t] = w_dkv h[t]          c_t = W_DKV h_t ([distaisys] sec. 2),
+ *                                       k^_t = W_KR h_t (the RoPE key projection)
+ *   k_t^R = RoPE(k^_t, pos[t])          decoupled RoPE key ([eyestech-pypi] item 2)
+ *   pool[page_table[seq_idx[t]][pos[t] / page]][pos[t] % page][:] = bf16([c_t || k_t^R])
+ * fp32 accumulation, one bf16 rounding per stored element.
+ *
+ *   h          device bf16 [n_tokens, d_model]
+ *   w_dkv      device bf16 [d_c + d_rope, d_model]; rows 0..d_c-1 = W_DKV, the rest W_KR
+ *   seq_idx    device int32 [n_tokens], each in [0, batch)
+ *   pos        device int32 [n_tokens], cache index = RoPE position, in [0, max_pages*page)
+ *   page_table device int32 [batch, max_pages]; physical page ids in [0, num_pages)
+ *   pool       device bf16 [num_pages, page_size, d_c + d_rope] (written in place)
+ *   dev_status device int32 word or NULL; device-side range errors land here
+ * Two tokens writing the same slot race (the caller must not do that).
+ * Returns MLA_OK or a negative mla_status.  n_tokens == 0 is a no-op.
+ */
+int mla_append_latent(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv,
+                      const int32_t* seq_idx, const int32_t* pos, const int32_t* page_table,
+                      int32_t batch, int32_t max_pages, mla_bf16* pool, int32_t num_pages,
+                      int32_t n_tokens, int32_t* dev_status, void* stream);
+
+/*
+ * mla_absorb_q - absorbed queries.
+ *
+ * For each token t and head h, with q[t][h] = [q_nope (qk_nope) || q_rope (d_rope)]:
+ *   q_lat[t][h][0 : d_c]        = W_UK,h^T q_nope   ([eyestech-blog] sec. 2;
+ *                                 [from-scratch] "Absorption, and why RoPE breaks it")
+ *   q_lat[t][h][d_c : d_c+d_rope] = RoPE(q_rope, pos[t])
+ * so that q_nope . (W_UK,h c) = q_lat[0:d_c] . c for every cached latent c.
+ *
+ *   q      device bf16 [n_tokens, H, qk_nope + d_rope]
+ *   pos    device int32 [n_tokens]; the query's own cache index (>= 0)
+ *   w_uk   device bf16 [H, qk_nope, d_c]   (w_uk[h] = W_UK,h, maps c to a key head)
+ *   q_lat  device bf16 [n_tokens, H, d_c + d_rope] (output)
+ * fp32 accumulation, bf16 output.  n_tokens == 0 is a no-op.
+ */
+int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
+                 const mla_bf16* w_uk, mla_bf16* q_lat, int32_t n_tokens, void* stream);
+
+/*
+ * mla_decode_workspace_bytes - device workspace mla_decode_attn needs for
+ * `batch` sequences with `nq` query tokens each, on the current device.
+ * Returns 0 for invalid arguments.
+ */
+size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t nq);
+
+/*
+ * mla_decode_attn - absorbed latent attention over the paged cache, then W_UV.
+ *
+ * Query token i (0 <= i < nq) of sequence b sits at cache index
+ * p = seq_lens[b] - nq + i and attends to cache indices 0..p (its own row, already
+ * appended, included; later tokens of the same step masked).  For head h with
+ * q_lat row [q~ || q_r] and cache row n = [c_n || k_n^R]:
+ *   s_n   = scale * (q~ . c_n + q_r . k_n^R)       content + positional score
+ *                                                  ([from-scratch], same section)
+ *   p     = softmax(s)                             scale = dims->softmax_scale or
+ *                                                  1/sqrt(qk_nope + d_rope)
+ *   o_lat = sum_n p_n c_n                          values read in latent space
+ *   out[b][i][h] = W_UV,h o_lat                    up-projected once ([from-scratch])
+ *   lse[b][i][h] = log sum_n exp(s_n)              natural log
+ * The key range of every sequence is cut into pages processed in parallel
+ * (split-KV); each part's softmax-normalised o_lat and lse go to the workspace
+ * and a combine step merges them with weights exp(lse_part - lse).
+ *
+ *   q_lat      device bf16 [batch, nq, H, d_c + d_rope] (as written by mla_absorb_q)
+ *   pool       device bf16 [num_pages, page_size, d_c + d_rope]
+ *   page_table device int32 [batch, max_pages]
+ *   seq_lens   device int32 [batch]: cache length after this step's append,
+ *              nq <= seq_lens[b] <= max_pages * page_size
+ *   w_uv       device bf16 [H, v_head, d_c]   (w_uv[h] = W_UV,h)
+ *   workspace  device scratch of ws_bytes >= mla_decode_workspace_bytes(...)
+ *   out        device bf16 [batch, nq, H, v_head] (output)
+ *   lse        device fp32 [batch, nq, H] (output) or NULL
+ *   dev_status device int32 word or NULL
+ * A sequence whose length is out of range gets zero output and lse = -inf; a
+ * page-table entry outside [0, num_pages) is skipped (never read).  Both record
+ * MLA_ERR_RANGE in dev_status.  batch <= 1024, nq <= 16.
+ */
+int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
+                    const int32_t* page_table, const int32_t* seq_lens, int32_t batch,
+                    int32_t nq, int32_t max_pages, int32_t num_pages, const mla_bf16* w_uv,
+                    void* workspace, size_t ws_bytes, mla_bf16* out, float* lse,
+                    int32_t* dev_status, void* stream);
+
+/* mla_status_read - wait for `stream`, then return the mla_status recorded in the
+ * device word dev_status (MLA_OK if none), or MLA_ERR_CUDA if the copy failed. */
+int mla_status_read(const int32_t* dev_status, void* stream);
+
+/* mla_status_clear - reset the device word to MLA_OK (asynchronous on stream). */
+int mla_status_clear(int32_t* dev_status, void* stream);
+
+/* mla_status_string - static description of an mla_status value. */
+const char* mla_status_string(int status);
+
+/* mla_version - library version string, e.g. "mla_b200 0.1.0 sm_100a". */
+const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H_ */

@@ -275,18 +275,22 @@ def decode_step(*, h, h_seq_idx, h_pos, q, q_pos, pool, page_table, lens, nq,
                 form="naive", heads=None, queries=None):
     """One decode step: append this step's cache rows, then attend.
 
-    1. rows = [W_DKV h_t || RoPE(W_KR h_t, pos_t)] written into a float64 copy
-       of the paged pool at (page_table[b][pos // page], pos % page).
+    1. rows = [W_DKV h_t || RoPE(W_KR h_t, pos_t)] become cache index pos_t of
+       sequence seq_idx_t ([songhuiming] "Update latent cache ... then up-project
+       ALL cached latents"; [eyestech-pypi] quickstart: the cache grows by one).
     2. For query token i of sequence b (cache index N_b - nq + i) and every head,
        attention over cache indices 0 .. N_b - nq + i (its own row included;
        the later query of the same step is masked: causal within the step).
+       Earlier rows are read from the paged pool through the page table.
        form="naive" decompresses K and V per head; form="absorbed" scores on
        latents with q~ = W_UK^T q_nope and up-projects o_lat once by W_UV.
-    `heads` (list of head indices) and `queries` (list of query-token indices)
-    restrict the attention to a sample; other entries of the outputs are NaN.
+    `pool` is anything indexable as pool[page_ids, slots] -> rows (only the rows
+    a query reads are widened to float64).  `heads` (head indices) and `queries`
+    (query-token indices) restrict the attention to a sample; other entries of
+    the outputs are NaN.
 
-    Returns dict(out [T, H, d_v], lse [T, H], pool (float64, after append),
-    q_lat [T, H, d_c + d_rope] (absorbed form only, else None)).
+    Returns dict(out [T, H, d_v], lse [T, H], rows [Ta, d_c + d_rope] (the
+    appended rows, float64), q_lat [T, H, d_c + d_rope] (absorbed form, else None)).
     """
     w_uk = np.asarray(w_uk, dtype=np.float64)
     w_uv = np.asarray(w_uv, dtype=np.float64)
@@ -296,9 +300,10 @@ def decode_step(*, h, h_seq_idx, h_pos, q, q_pos, pool, page_table, lens, nq,
     d_r = q.shape[-1] - d_h
     if scale is None:
         scale = softmax_scale(d_h, d_r)
-    pool = np.array(pool, dtype=np.float64)
     rows = kv_rows(h, w_dkv, np.asarray(h_pos), d_c, theta)
-    append_rows(pool, page_table, h_seq_idx, h_pos, rows)
+    appended = {}                                   # sequence -> {cache index: row}
+    for t in range(len(h_pos)):
+        appended.setdefault(int(h_seq_idx[t]), {})[int(h_pos[t])] = rows[t]
 
     T = q.shape[0]
     heads = list(range(H)) if heads is None else list(heads)
@@ -311,7 +316,10 @@ def decode_step(*, h, h_seq_idx, h_pos, q, q_pos, pool, page_table, lens, nq,
         p = int(q_pos[t])
         n = p + 1                                   # keys 0 .. p are visible
         assert n <= int(lens[b])
-        cache = gather_cache(pool, page_table[b], n)
+        cache = np.asarray(gather_cache(pool, page_table[b], n), dtype=np.float64)
+        for idx, row in appended.get(b, {}).items():
+            if idx < n:
+                cache[idx] = row
         C, KR = cache[:, :d_c], cache[:, d_c:]
         if form == "naive":
             o, l = attend_naive(q[t, heads], p, C, KR, w_uk[heads], w_uv[heads], scale, theta)
@@ -321,7 +329,7 @@ def decode_step(*, h, h_seq_idx, h_pos, q, q_pos, pool, page_table, lens, nq,
             raise ValueError(form)
         out[t, heads] = o
         lse[t, heads] = l
-    return {"out": out, "lse": lse, "pool": pool, "q_lat": q_lat}
+    return {"out": out, "lse": lse, "rows": rows, "q_lat": q_lat}
 
 
 def attend_paged_latents(*, q_lat, pool, page_table, lens, nq, w_uv, scale,

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/mla.h declares, and rejects bad arguments before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import head_latent_attention_07_b200 as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\**\s*(mla_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(M.LIB_PATH):
+        from head_latent_attention_07_b200 import build
+        build.build()
+    return M.load_library()
+
+
+def test_header_declares_the_three_calls():
+    names = declared_entry_points()
+    for n in ("mla_append_latent", "mla_absorb_q", "mla_decode_attn"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_entry_points()
+    assert names, "no entry points parsed from include/mla.h"
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/mla.h but not exported"
+    # and the binding declares a signature for every one of them
+    assert sorted(M.SIGNATURES) == names
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in M.version()
+    for code in range(0, -8, -1):
+        s = M.status_string(code)
+        assert s.startswith("MLA_"), s
+    assert M.status_string(-99) == "unknown mla_status"
+
+
+def v3_dims(**kw):
+    d = dict(n_heads=128, d_c=512, d_rope=64, qk_nope=128, v_head=128, d_model=7168, page_size=64,
+             softmax_scale=0.0, rope_theta=0.0)
+    d.update(kw)
+    return M.MlaDims(**d)
+
+
+FAKE = 1 << 20          # 16-byte aligned fake device address (never dereferenced)
+FAKE_MIS = FAKE + 2     # misaligned
+
+
+def absorb(lib, dims, q=FAKE, pos=FAKE, w=FAKE, out=FAKE, n=4):
+    return lib.mla_absorb_q(ctypes.byref(dims) if dims is not None else None, q, pos, w, out, n, None)
+
+
+def test_absorb_argument_checks(lib):
+    assert absorb(lib, None) == M.MLA_ERR_INVALID_ARG
+    assert absorb(lib, v3_dims(d_rope=0)) == M.MLA_ERR_UNSUPPORTED     # no decoupled RoPE: refuse
+    assert absorb(lib, v3_dims(n_heads=129)) == M.MLA_ERR_UNSUPPORTED
+    assert absorb(lib, v3_dims(d_c=520 + 8)) == M.MLA_ERR_UNSUPPORTED
+    assert absorb(lib, v3_dims(d_c=500)) == M.MLA_ERR_UNSUPPORTED
+    assert absorb(lib, v3_dims(n_heads=0)) == M.MLA_ERR_INVALID_ARG
+    assert absorb(lib, v3_dims(softmax_scale=float("nan"))) == M.MLA_ERR_INVALID_ARG
+    assert absorb(lib, v3_dims(), q=None) == M.MLA_ERR_INVALID_ARG
+    assert absorb(lib, v3_dims(), q=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert absorb(lib, v3_dims(), n=-1) == M.MLA_ERR_INVALID_ARG
+    assert absorb(lib, v3_dims(), q=None, n=0) == M.MLA_OK              # empty: no-op
+
+
+def test_append_argument_checks(lib):
+    d = v3_dims()
+    call = lambda **kw: lib.mla_append_latent(
+        ctypes.byref(d), kw.get("h", FAKE), FAKE, FAKE, FAKE, FAKE, kw.get("B", 2), kw.get("mp", 4),
+        kw.get("pool", FAKE), kw.get("np_", 8), kw.get("T", 2), kw.get("st", None), None)
+    assert call(h=None) == M.MLA_ERR_INVALID_ARG
+    assert call(pool=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(st=FAKE + 4) == M.MLA_ERR_MISALIGNED
+    assert call(B=0) == M.MLA_ERR_INVALID_ARG
+    assert call(np_=0) == M.MLA_ERR_INVALID_ARG
+    assert call(T=0, h=None) == M.MLA_OK
+
+
+def test_decode_argument_checks(lib):
+    d = v3_dims()
+    def call(**kw):
+        return lib.mla_decode_attn(
+            ctypes.byref(d), kw.get("q", FAKE), FAKE, FAKE, FAKE, kw.get("B", 2), kw.get("nq", 1),
+            kw.get("mp", 4), 8, FAKE, kw.get("ws", FAKE), kw.get("wsb", 1 << 30), kw.get("out", FAKE),
+            kw.get("lse", None), None, None)
+    assert call(q=None) == M.MLA_ERR_INVALID_ARG
+    assert call(ws=None) == M.MLA_ERR_INVALID_ARG
+    assert call(B=0) == M.MLA_ERR_INVALID_ARG
+    assert call(nq=0) == M.MLA_ERR_INVALID_ARG
+    assert call(B=1025) == M.MLA_ERR_UNSUPPORTED
+    assert call(nq=17) == M.MLA_ERR_UNSUPPORTED
+    assert call(mp=1 << 26) == M.MLA_ERR_UNSUPPORTED       # max_pages * page overflows int32
+    assert call(out=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(lse=FAKE + 4) == M.MLA_ERR_MISALIGNED
+
+
+def test_workspace_query_rejects_bad_arguments(lib):
+    assert lib.mla_decode_workspace_bytes(ctypes.byref(v3_dims()), 0, 1) == 0
+    assert lib.mla_decode_workspace_bytes(ctypes.byref(v3_dims()), 1, 0) == 0
+    assert lib.mla_decode_workspace_bytes(ctypes.byref(v3_dims(d_rope=0)), 1, 1) == 0
+    assert lib.mla_decode_workspace_bytes(None, 1, 1) == 0
+
+
+def test_status_calls_reject_null(lib):
+    assert lib.mla_status_read(None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_status_clear(None, None) == M.MLA_ERR_INVALID_ARG

@@ -291,8 +291,10 @@ def test_decode_step_matches_paged_latent_attention():
     r = O.decode_step(h=f("h"), h_seq_idx=x.h_seq_idx, h_pos=x.h_pos, q=f("q"), q_pos=x.pos,
                       pool=f("pool"), page_table=x.page_table, lens=x.lens, nq=1,
                       w_dkv=f("w_dkv"), w_uk=f("w_uk"), w_uv=f("w_uv"), d_c=w.d_c)
+    pool = f("pool")
+    O.append_rows(pool, x.page_table, x.h_seq_idx, x.h_pos, r["rows"])   # write, then read back
     q_lat = O.absorb_queries(f("q"), x.pos, f("w_uk"))
-    o, l = O.attend_paged_latents(q_lat=q_lat, pool=r["pool"], page_table=x.page_table, lens=x.lens,
+    o, l = O.attend_paged_latents(q_lat=q_lat, pool=pool, page_table=x.page_table, lens=x.lens,
                                   nq=1, w_uv=f("w_uv"), scale=O.softmax_scale(8, 8))
     assert np.abs(o - r["out"]).max() <= 1e-12
     assert np.abs(l - r["lse"]).max() <= 1e-12

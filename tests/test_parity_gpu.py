@@ -1,0 +1,196 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+identical seeded inputs.
+
+Floating outputs (out, lse, q_lat, appended cache rows) must agree within max
+abs <= 2e-2 and relative L2 <= 1e-2; paging is bit-exact (every slot the step
+does not write keeps its bytes, canary pages included).  Sizes span several
+pages and split pieces with ragged tails; the full-size workloads are checked on
+sampled heads and queries, in the launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workload as W
+from oracle import mla as O
+from mla_gpu_util import GpuStep, assert_close, bits_of, dims_of, f64_of, oracle_inputs, dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+class Bf16Pool:
+    """Read-only view of a bf16 pool that widens only the rows the oracle gathers."""
+
+    def __init__(self, bits):
+        self.bits = bits
+        self.shape = bits.shape
+
+    def __getitem__(self, idx):
+        return W.bf16_to_f32(self.bits[idx])
+
+
+def check_step(x, g, heads=None, queries=None, form="naive"):
+    w = x.workload
+    T, H = w.tokens, w.n_heads
+    args = oracle_inputs(x)
+    args["pool"] = Bf16Pool(x.bits["pool"])
+    ref = O.decode_step(**args, form=form, heads=heads, queries=queries)
+    out = f64_of(g.out).reshape(T, H, w.v_head)
+    lse = f64_of(g.lse).reshape(T, H)
+    hs = list(range(H)) if heads is None else list(heads)
+    qs = list(range(T)) if queries is None else list(queries)
+    sel = np.ix_(qs, hs)
+    assert_close(out[sel], ref["out"][sel], "out")
+    assert_close(lse[sel], ref["lse"][sel], "lse")
+    # absorbed queries, all of them
+    ql_ref = O.absorb_queries(x.f64("q"), x.pos, x.f64("w_uk"))
+    assert_close(f64_of(g.q_lat), ql_ref, "q_lat")
+    check_pool(x, g, ref["rows"])
+    return ref
+
+
+def check_pool(x, g, rows_ref):
+    """Appended rows land in their slots (values within tolerance); every other
+    slot is bit-identical to the input pool."""
+    P = x.workload.page_size
+    got = bits_of(g.pool)
+    before = x.bits["pool"]
+    pages = x.page_table[x.h_seq_idx, x.h_pos // P]
+    slots = x.h_pos % P
+    assert_close(W.bf16_to_f32(got[pages, slots]).astype(np.float64), rows_ref, "appended rows")
+    mask = np.ones(before.shape[:2], dtype=bool)
+    mask[pages, slots] = False
+    assert np.array_equal(got[mask], before[mask]), "a slot outside this step's rows changed"
+
+
+def test_tiny_workload_end_to_end():
+    x = W.make_decode_inputs(W.WORKLOADS["tiny"], seed=0, append_all=True)
+    g = GpuStep(x).run()
+    assert g.device_status() == 0
+    check_step(x, g)
+    check_step(x, g, form="absorbed")
+
+
+def test_v2_workload_end_to_end():
+    x = W.make_decode_inputs(W.WORKLOADS["v2"], seed=0)
+    g = GpuStep(x).run()
+    assert g.device_status() == 0
+    check_step(x, g)
+
+
+SMALL = dict(n_heads=8, d_model=256, d_c=512, d_rope=64, qk_nope=128, v_head=128)
+
+
+@pytest.mark.parametrize("nq,lens", [
+    (1, [1]), (1, [63]), (1, [64]), (1, [65]), (1, [1, 64, 65, 128, 129, 300, 1000, 4097]),
+    (2, [2, 3, 64, 65, 66, 127, 128, 129]), (2, [5000, 2, 7, 4096, 63]),
+])
+def test_ragged_lengths_and_pieces(nq, lens):
+    w = W.Workload("ragged_small", batch=len(lens), nq=nq, context=None, ragged=(1, 1), **SMALL)
+    x = W.make_decode_inputs(w, seed=11, spare_pages=3, lens=lens)
+    g = GpuStep(x).run()
+    assert g.device_status() == 0
+    check_step(x, g)
+
+
+def test_decode_only_with_peaked_scores():
+    # q_lat drawn directly; some keys planted along q~ so the running max jumps late
+    w = W.Workload("peaked", batch=3, nq=1, context=3000, **SMALL)
+    x = W.make_decode_inputs(w, seed=21)
+    rng = np.random.default_rng(5)
+    q_lat = rng.standard_normal((w.tokens, w.n_heads, w.row)).astype(np.float32)
+    pool = W.bf16_to_f32(x.bits["pool"]).copy()
+    for b in range(w.batch):
+        for n in (17, 1500, 2999):                      # late keys with large scores
+            pg, sl = x.page_table[b, n // 64], n % 64
+            pool[pg, sl, :w.d_c] = q_lat[b * w.nq, 0, :w.d_c]
+    x.bits["pool"] = W.bf16_bits(pool)
+    ql_bits = W.bf16_bits(q_lat)
+    g = GpuStep(x)
+    ql_dev = dev_bf16(ql_bits)
+    g.decode(ql_dev)
+    torch.cuda.synchronize()
+    assert g.device_status() == 0
+    ref_o, ref_l = O.attend_paged_latents(q_lat=W.bf16_to_f32(ql_bits), pool=Bf16Pool(x.bits["pool"]),
+                                          page_table=x.page_table, lens=x.lens, nq=1, w_uv=x.f64("w_uv"),
+                                          scale=O.softmax_scale(w.qk_nope, w.d_rope))
+    assert_close(f64_of(g.out).reshape(ref_o.shape), ref_o, "out")
+    assert_close(f64_of(g.lse).reshape(ref_l.shape), ref_l, "lse")
+    assert np.abs(ref_l).max() > 20        # the plants really dominate
+
+
+def test_invalid_page_id_is_recorded_not_read():
+    w = W.Workload("badpage", batch=2, nq=1, context=200, **SMALL)
+    x = W.make_decode_inputs(w, seed=3)
+    g = GpuStep(x)
+    g.append()
+    g.absorb()
+    torch.cuda.synchronize()
+    assert g.device_status() == 0
+    pt = x.page_table.copy()
+    pt[1, 1] = x.num_pages + 1000                     # sequence 1's second page: out of range
+    g.page_table.copy_(torch.from_numpy(pt))
+    g.decode()
+    torch.cuda.synchronize()
+    assert g.device_status() == -7                    # MLA_ERR_RANGE
+    out = f64_of(g.out)
+    assert np.isfinite(out).all()
+
+
+def test_out_of_range_length_gives_zero_and_neg_inf():
+    w = W.Workload("badlen", batch=3, nq=1, context=130, **SMALL)
+    x = W.make_decode_inputs(w, seed=4)
+    g = GpuStep(x)
+    g.append()
+    g.absorb()
+    lens = x.lens.copy()
+    lens[1] = x.page_table.shape[1] * 64 + 1            # longer than its page-table row
+    g.seq_lens.copy_(torch.from_numpy(lens))
+    g.decode()
+    torch.cuda.synchronize()
+    assert g.device_status() == -7
+    out, lse = f64_of(g.out), f64_of(g.lse)
+    assert (out[1] == 0).all() and np.isneginf(lse[1]).all()
+    # the other sequences are unaffected
+    args = oracle_inputs(x)
+    args["pool"] = Bf16Pool(x.bits["pool"])
+    ref = O.decode_step(**args, form="absorbed", queries=[0, 2])
+    assert_close(out.reshape(3, -1, 128)[[0, 2]], ref["out"][[0, 2]], "out")
+
+
+def test_status_clear_and_read():
+    st = torch.zeros(4, dtype=torch.int32, device="cuda")
+    st[0] = -7
+    import head_latent_attention_07_b200 as M
+    assert M.mla_status_read(st) == -7
+    M.mla_status_clear(st)
+    assert M.mla_status_read(st) == 0
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+
+def _sampled(name, heads, queries, naive_pairs):
+    x = W.make_decode_inputs(W.WORKLOADS[name], seed=0)
+    g = GpuStep(x).run()
+    assert g.device_status() == 0
+    w = x.workload
+    check_step(x, g, heads=heads, queries=queries, form="absorbed")
+    # the naive (decompressing) form on a few (query, head) pairs
+    args = oracle_inputs(x)
+    args["pool"] = Bf16Pool(x.bits["pool"])
+    out = f64_of(g.out).reshape(w.tokens, w.n_heads, w.v_head)
+    for t, h in naive_pairs:
+        ref = O.decode_step(**args, heads=[h], queries=[t])
+        assert_close(out[t, h], ref["out"][t, h], f"out naive ({t},{h})")
+
+
+def test_v3_full_size_sampled():
+    _sampled("v3", heads=[0, 1, 63, 127], queries=None, naive_pairs=[(0, 0), (15, 127)])
+
+
+def test_long_context_full_size_sampled():
+    _sampled("long", heads=[0, 77, 127], queries=None, naive_pairs=[(7, 3)])
+
+
+def test_ragged_serving_full_size_sampled():
+    _sampled("ragged", heads=[0, 64, 127], queries=[0, 1, 2, 3, 50, 51, 126, 127], naive_pairs=[(1, 5)])

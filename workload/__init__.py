@@ -105,15 +105,26 @@ def _normal(seed: int, name: str, shape, std: float = 1.0) -> np.ndarray:
 
 
 def _normal_bf16(seed: int, name: str, shape, chunk: int = 1 << 22) -> np.ndarray:
-    """N(0,1) draws rounded to bf16, produced chunk by chunk (bounded host memory
-    for the large latent-cache pools).  Same values as bf16_bits(_normal(...))."""
-    g = rng_for(seed, name)
+    """N(0,1) draws rounded to bf16 for the large latent-cache pools.
+
+    The tensor is cut into chunks of `chunk` elements; chunk k draws from its own
+    PCG64 stream keyed by (seed, name, k), so the values do not depend on how many
+    threads fill them (numpy releases the GIL while it draws).
+    """
+    import concurrent.futures
+    import os
     out = np.empty(int(np.prod(shape)), dtype=np.uint16)
-    buf = np.empty(chunk, dtype=np.float32)
-    for s in range(0, out.size, chunk):
+    key = zlib.crc32(name.encode())
+
+    def fill(k):
+        s = k * chunk
         n = min(chunk, out.size - s)
-        g.standard_normal(out=buf[:n], dtype=np.float32)
-        out[s:s + n] = bf16_bits(buf[:n])
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, key, k])))
+        out[s:s + n] = bf16_bits(g.standard_normal(size=n, dtype=np.float32))
+
+    nchunks = (out.size + chunk - 1) // chunk
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(nchunks)))
     return out.reshape(shape)
 
 
@@ -174,7 +185,7 @@ class DecodeInputs:
 
 def make_decode_inputs(w: Workload, seed: int = 0, spare_pages: int = 0,
                        prefill: bool = True, max_pages: int | None = None,
-                       append_all: bool = False) -> DecodeInputs:
+                       append_all: bool = False, lens=None) -> DecodeInputs:
     """Draw every input of one decode step of workload `w`.
 
     Tensors (bf16 bits):
@@ -189,8 +200,10 @@ def make_decode_inputs(w: Workload, seed: int = 0, spare_pages: int = 0,
     By default the appended tokens are the query tokens (Ta = T).  With
     `append_all` every cache row of every sequence is appended this step
     (Ta = sum N_b, pool starts zeroed): the tiny case builds its whole cache so.
+    `lens` overrides the per-sequence context lengths of the workload.
     """
-    lens = context_lengths(w, seed)
+    lens = context_lengths(w, seed) if lens is None else np.asarray(lens, dtype=np.int32)
+    assert lens.shape == (w.batch,) and (lens >= w.nq).all()
     T = w.tokens
     seq_idx = np.repeat(np.arange(w.batch, dtype=np.int32), w.nq)
     pos = (lens[seq_idx] - w.nq + np.tile(np.arange(w.nq, dtype=np.int32), w.batch)).astype(np.int32)
