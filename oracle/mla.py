@@ -339,7 +339,6 @@ def attend_paged_latents(*, q_lat, pool, page_table, lens, nq, w_uv, scale,
     b = t // nq sits at cache index N_b - nq + t % nq and sees indices up to it.
     Returns out [T, H, d_v] and lse [T, H] (NaN outside the sample)."""
     q_lat = np.asarray(q_lat, dtype=np.float64)
-    pool = np.asarray(pool)
     T, H = q_lat.shape[0], q_lat.shape[1]
     d_c = np.asarray(w_uv).shape[2]
     d_v = np.asarray(w_uv).shape[1]
