@@ -38,6 +38,7 @@ SIGNATURES = {
     "mla_decode_workspace_bytes": (ctypes.c_size_t, [_P, _I, _I]),
     "mla_decode_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, ctypes.c_size_t,
                                        _P, _P, _P, _P]),
+    "mla_decode_attn_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "mla_status_read": (ctypes.c_int, [_P, _P]),
     "mla_status_clear": (ctypes.c_int, [_P, _P]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -203,6 +204,31 @@ def mla_decode_attn(dims: MlaDims, q_lat, pool, page_table, seq_lens, w_uv, work
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
         _ptr(dev_status, torch.int32, "dev_status"), _stream(stream))
     _check(st, "mla_decode_attn")
+
+
+def mla_decode_attn_noalloc(dims: MlaDims, q_lat, pool, page_table, seq_lens, w_uv, out,
+                            lse=None, dev_status=None, stream=None) -> None:
+    """mla_decode_attn without a caller workspace: the library's own 64 MiB device
+    scratch is used instead (see include/mla.h for the sharing rules)."""
+    torch = _torch()
+    B, nq = q_lat.shape[0], q_lat.shape[1]
+    _shape(q_lat, (B, nq, dims.n_heads, dims.row), "q_lat")
+    num_pages = pool.shape[0]
+    _shape(pool, (num_pages, dims.page_size, dims.row), "pool")
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, max_pages]")
+    _shape(seq_lens, (B,), "seq_lens")
+    _shape(w_uv, (dims.n_heads, dims.v_head, dims.d_c), "w_uv")
+    _shape(out, (B, nq, dims.n_heads, dims.v_head), "out")
+    if lse is not None:
+        _shape(lse, (B, nq, dims.n_heads), "lse")
+    st = load_library().mla_decode_attn_noalloc(
+        ctypes.byref(dims), _ptr(q_lat, torch.bfloat16, "q_lat"), _ptr(pool, torch.bfloat16, "pool"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        B, nq, page_table.shape[1], num_pages, _ptr(w_uv, torch.bfloat16, "w_uv"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(dev_status, torch.int32, "dev_status"), _stream(stream))
+    _check(st, "mla_decode_attn_noalloc")
 
 
 def mla_status_read(dev_status, stream=None) -> int:

@@ -168,6 +168,35 @@ int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16*
                     void* workspace, size_t ws_bytes, mla_bf16* out, float* lse,
                     int32_t* dev_status, void* stream);
 
+/*
+ * mla_decode_attn_noalloc - mla_decode_attn for callers that cannot allocate.
+ *
+ * The pages describe no such call; it exists for deployment.  Some callers
+ * cannot give mla_decode_attn a workspace: code that runs inside a host framework
+ * which owns all device memory (a serving-engine plugin with a fixed memory
+ * budget, where only the framework allocates), or a latency-critical decode loop
+ * that must not call cudaMalloc because it can synchronise the device.  This call
+ * computes exactly what mla_decode_attn computes (same arguments minus the
+ * workspace) and allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ * library routine.
+ *
+ * Scratch: a 64 MiB device array owned by the library.  Every GPU that loads the
+ * library holds one copy until the process exits.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.
+ * Limit: a call whose mla_decode_workspace_bytes(dims, batch, nq) exceeds 64 MiB
+ * returns MLA_ERR_WORKSPACE without launching anything.
+ * Sharing: all calls on a device use the same array, which keeps the last call's
+ * contents.  Nothing in it needs to start at zero.  Calls that overlap on the GPU
+ * (on different streams, or from several host threads) race on the array and
+ * corrupt each other's results: issue them one after another on one stream.
+ * Other arguments, outputs and errors: as for mla_decode_attn.
+ */
+int mla_decode_attn_noalloc(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
+                            const int32_t* page_table, const int32_t* seq_lens, int32_t batch,
+                            int32_t nq, int32_t max_pages, int32_t num_pages, const mla_bf16* w_uv,
+                            mla_bf16* out, float* lse, int32_t* dev_status, void* stream);
+
 /* mla_status_read - wait for `stream`, then return the mla_status recorded in the
  * device word dev_status (MLA_OK if none), or MLA_ERR_CUDA if the copy failed. */
 int mla_status_read(const int32_t* dev_status, void* stream);
