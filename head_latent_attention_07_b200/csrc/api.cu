@@ -139,11 +139,17 @@ int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16*
   a.batch = batch; a.nq = nq; a.n_heads = dims->n_heads; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
   a.v_head = dims->v_head; a.page_size = dims->page_size; a.max_pages = max_pages;
   a.num_pages = num_pages; a.scale = eff_scale(dims);
-  const int groups = mla::decode_simt_row_groups(nq * dims->n_heads);
-  int G = (2 * sms + groups - 1) / groups;
-  a.G = G < 1 ? 1 : (G > sms ? sms : G);
   cudaStream_t s = (cudaStream_t)stream;
-  if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
+  if (mla::decode_tc_supported(dims->d_c, dims->d_rope, dims->page_size)) {
+    // tensor-core path: one CTA pair per worker and 128-row tile
+    a.G = mla::decode_tc_workers(sms, nq * dims->n_heads);
+    if ((st = cuda_status(mla::launch_decode_split_tc(a, mla::kSpinLimitCycles, s))) != MLA_OK) return st;
+  } else {
+    const int groups = mla::decode_simt_row_groups(nq * dims->n_heads);
+    int G = (2 * sms + groups - 1) / groups;
+    a.G = G < 1 ? 1 : (G > sms ? sms : G);
+    if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
+  }
   return cuda_status(mla::launch_decode_combine(a, s));
 }
 

@@ -48,6 +48,12 @@ size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);
 int decode_simt_row_groups(int rows_total);
 cudaError_t launch_decode_split_simt(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream);
+
+// Tensor-core split kernel (d_c = 512, d_rope = 64, 64-token pages).
+bool decode_tc_supported(int d_c, int d_rope, int page_size);
+int decode_tc_workers(int sms, int rows_total);
+cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cudaStream_t stream);
+constexpr long long kSpinLimitCycles = 1ll << 31;  // ~1 s at B200 clocks per bounded wait
 cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
 

@@ -1,0 +1,522 @@
+// Split-KV latent attention on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// Shape: d_c = 512, d_rope = 64 (576-wide cache rows), 64-token pages, up to 128
+// query rows (query token, head) per tile.
+//
+// A CTA pair (cluster of 2) works on one (worker, row tile).  CTA c owns latent
+// columns [256c, 256c + 256) and RoPE columns [512 + 32c, 512 + 32c + 32) of
+// every cache row and of the query tile, so each page is read from HBM once per
+// pair, half by each CTA.  Per page (64 tokens):
+//   GEMM1   S_c[128 x 64]  = Q_c[128 x 288] . K_c[64 x 288]^T        (tcgen05, TMEM)
+//   swap    each CTA scales S_c to log2 units, rounds it to fp16 and stores it
+//           into its peer's shared memory (st.async); both CTAs then hold the same
+//           S = fp16(S_0) + fp16(S_1), the full 576-wide score (content + RoPE)
+//   softmax one thread per query row: running max / sum over the page, P in bf16
+//   GEMM2   O_c[128 x 256] += P[128 x 64] . C_c[64 x 256]               (tcgen05, TMEM)
+// Both CTAs compute the same softmax, so the two O halves share one normaliser.
+// The running max is only moved (and O rescaled in TMEM) when it grows by more
+// than 2^8; otherwise P is taken relative to the stale max (P <= 256).
+// TMEM: O_c uses columns [0, 256), the two S buffers [256, 320) and [320, 384).
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA loads (query tile once per
+// piece, pages into a 3-stage ring), warp 1 owns TMEM and lane 0 issues the MMAs,
+// warps 2..5 (one per TMEM lane quarter) run the exchange, softmax and epilogue.
+// Every mbarrier wait is bounded: on time-out the kernel records MLA_ERR_TIMEOUT,
+// stops its loops, drains its own copies and MMAs and frees TMEM.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.h"
+#include "plan.cuh"
+#include "sm100.cuh"
+
+namespace mla {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr int kQBytes = 4 * 16384 + 8192;     // 4 latent blocks [128 x 64] + RoPE block [128 x 32]
+constexpr int kPageBytes = 4 * 8192 + 4096;   // 4 latent blocks [64 x 64]  + RoPE block [64 x 32]
+constexpr int kXBytes = 128 * 128;            // [128 rows x 64] fp16 scores, then bf16 P
+constexpr int kOffQ = 0;
+constexpr int kOffPg = kOffQ + kQBytes;
+constexpr int kOffX = kOffPg + kStages * kPageBytes;
+constexpr int kOffPlan = kOffX + 2 * kXBytes;
+constexpr int kOffBar = kOffPlan + ((int(sizeof(PlanSmem)) + 127) & ~127);
+constexpr int kNumBars = 24;
+constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 64 + 1024;  // + misc + 1 KB alignment slack
+constexpr float kRescaleThreshold = 8.0f;     // log2 units: rescale when the max grows by > 2^8
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS = 256;              // first S buffer column
+
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffPg % 1024 == 0 && kPageBytes % 1024 == 0 && kOffX % 1024 == 0, "swizzle alignment");
+
+struct TcParams {
+  DecodeArgs d;
+  int rows_total;   // nq * H
+  float scale_log2; // softmax scale * log2(e)
+  long long spin_limit;
+};
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t pg_full[kStages], pg_empty[kStages];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t x_full[2], x_free[2];
+  uint64_t p_full[2], o_done[2];
+  uint64_t o_free, drain;
+};
+static_assert(sizeof(Bars) <= kNumBars * 8, "barrier area");
+
+// One (sequence, page range) overlap of this worker's chunk.
+struct Piece {
+  int b, pg_begin, pg_end, id;
+};
+
+// Iterates the pieces of worker w in order; identical in every role.
+struct PieceIter {
+  const PlanSmem* ps;
+  int batch, w, chunk, f, f1, b;
+  __device__ PieceIter(const PlanSmem* ps_, int batch_, int w_) : ps(ps_), batch(batch_), w(w_) {
+    chunk = ps->chunk;
+    const int total = ps->start[batch];
+    f = w * chunk;
+    f1 = min(f + chunk, total);
+    b = f < f1 ? seq_of_flat_page(ps, batch, f) : 0;
+  }
+  __device__ bool next(Piece* p) {
+    if (f >= f1) return false;
+    while (ps->start[b + 1] <= f) ++b;
+    const int sb = ps->start[b];
+    const int e = min(f1, ps->start[b + 1]);
+    p->b = b;
+    p->pg_begin = f - sb;
+    p->pg_end = e - sb;
+    p->id = ps->piece_begin[b] + (w - sb / chunk);
+    f = e;
+    return true;
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_half2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<__half2*>(&v));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_constant__ CUtensorMap tq64,
+                       const __grid_constant__ CUtensorMap tp128, const __grid_constant__ CUtensorMap tp64,
+                       const TcParams prm) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* q_s = sm + kOffQ;
+  unsigned char* pg_s = sm + kOffPg;
+  unsigned char* x_s = sm + kOffX;
+  PlanSmem* plan = reinterpret_cast<PlanSmem*>(sm + kOffPlan);
+  Bars* bar = reinterpret_cast<Bars*>(sm + kOffBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + kOffBar + kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffBar + kNumBars * 8 + 16);
+
+  const DecodeArgs& a = prm.d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t c = cluster_ctarank();
+  const uint32_t peer = c ^ 1u;
+  const int w = blockIdx.x >> 1;
+  const int row0 = blockIdx.y * 128;
+  const int rows_valid = min(128, prm.rows_total - row0);
+  const long long lim = prm.spin_limit;
+  int32_t* status = a.dev_status;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_empty, 1);
+    for (int s = 0; s < kStages; ++s) { mbar_init(&bar->pg_full[s], 1); mbar_init(&bar->pg_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->s_full[s], 1);
+      mbar_init(&bar->s_empty[s], 4);
+      mbar_init(&bar->x_full[s], 1);
+      mbar_init(&bar->x_free[s], 1);
+      mbar_init(&bar->p_full[s], 4);
+      mbar_init(&bar->o_done[s], 1);
+    }
+    mbar_init(&bar->o_free, 4);
+    mbar_init(&bar->drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tq128); tma_prefetch(&tq64); tma_prefetch(&tp128); tma_prefetch(&tp64);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  build_plan(plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G,
+             (blockIdx.x == 0 && blockIdx.y == 0) ? status : nullptr);  // ends with __syncthreads
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised before any remote traffic
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      PieceIter it(plan, a.batch, w);
+      Piece pc;
+      int j = 0, p = 0;
+      int issued[kStages] = {0, 0, 0}, issued_q = 0;
+      while (!*abort_flag && it.next(&pc)) {
+        if (p > 0 && !mbar_wait(&bar->q_empty, (p - 1) & 1, abort_flag, status, lim)) break;
+        ++issued_q;
+        const int qrow = pc.b * prm.rows_total + row0;
+        mbar_arrive_expect_tx(&bar->q_full, kQBytes);
+        for (int i = 0; i < 4; ++i) tma_load_2d(q_s + i * 16384, &tq128, c * 256 + 64 * i, qrow, &bar->q_full);
+        tma_load_2d(q_s + 65536, &tq64, 512 + 32 * c, qrow, &bar->q_full);
+        bool ok = true;
+        for (int pg = pc.pg_begin; pg < pc.pg_end; ++pg, ++j) {
+          const int st = j % kStages;
+          if (j >= kStages && !mbar_wait(&bar->pg_empty[st], ((j / kStages) - 1) & 1, abort_flag, status, lim)) {
+            ok = false;
+            break;
+          }
+          int id = a.page_table[(size_t)pc.b * a.max_pages + pg];
+          if (id < 0 || id >= a.num_pages) id = 0;  // never read: the softmax masks and zeroes it
+          unsigned char* dst = pg_s + st * kPageBytes;
+          mbar_arrive_expect_tx(&bar->pg_full[st], kPageBytes);
+          for (int i = 0; i < 4; ++i) tma_load_2d(dst + i * 8192, &tp128, c * 256 + 64 * i, id * 64, &bar->pg_full[st]);
+          tma_load_2d(dst + 32768, &tp64, 512 + 32 * c, id * 64, &bar->pg_full[st]);
+          ++issued[st];
+        }
+        if (!ok) break;
+        ++p;
+      }
+      if (*abort_flag) {
+        // copies still in flight must land before this CTA's shared memory is released
+        for (int s = 0; s < kStages; ++s)
+          if (issued[s] > 0) mbar_wait_drain(&bar->pg_full[s], (issued[s] - 1) & 1, lim);
+        if (issued_q > 0) mbar_wait_drain(&bar->q_full, (issued_q - 1) & 1, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id1 = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t id2 = idesc_bf16_f32(128, 256, 0, 1);
+      PieceIter it(plan, a.batch, w);
+      Piece pc;
+      int j = 0, p = 0;
+      bool ok = true;
+      auto gemm2 = [&](int jj, bool first) -> bool {
+        if (first && p > 0 && !mbar_wait(&bar->o_free, (p - 1) & 1, abort_flag, status, lim)) return false;
+        if (!mbar_wait(&bar->p_full[jj & 1], (jj >> 1) & 1, abort_flag, status, lim)) return false;
+        tc_fence_after();
+        const uint32_t xa = smem_u32(x_s + (jj & 1) * kXBytes);
+        const uint32_t pb = smem_u32(pg_s + (jj % kStages) * kPageBytes);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t da = smem_desc(xa + ks * 32, 16, 1024, kSwizzle128);
+          const uint64_t db = smem_desc(pb + ks * 2048, 8192, 1024, kSwizzle128);
+          mma_bf16(tmem, da, db, id2, (first && ks == 0) ? 0u : 1u);
+        }
+        mma_commit(&bar->pg_empty[jj % kStages]);
+        mma_commit(&bar->o_done[jj & 1]);
+        mma_commit_mc(&bar->x_free[jj & 1], uint16_t(1u << peer));
+        return true;
+      };
+      while (ok && it.next(&pc)) {
+        const int n = pc.pg_end - pc.pg_begin;
+        if (!mbar_wait(&bar->q_full, p & 1, abort_flag, status, lim)) break;
+        const uint32_t qa = smem_u32(q_s);
+        for (int k = 0; k < n && ok; ++k) {
+          const int jj = j + k;
+          const int st = jj % kStages;
+          if (!mbar_wait(&bar->pg_full[st], (jj / kStages) & 1, abort_flag, status, lim) ||
+              (jj >= 2 && !mbar_wait(&bar->s_empty[jj & 1], ((jj >> 1) - 1) & 1, abort_flag, status, lim))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pb = smem_u32(pg_s + st * kPageBytes);
+          const uint32_t ts = tmem + kTmemS + 64 * (jj & 1);
+#pragma unroll
+          for (int ks = 0; ks < 18; ++ks) {
+            uint64_t da, db;
+            if (ks < 16) {
+              da = smem_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128);
+              db = smem_desc(pb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128);
+            } else {
+              da = smem_desc(qa + 65536 + (ks - 16) * 32, 16, 512, kSwizzle64);
+              db = smem_desc(pb + 32768 + (ks - 16) * 32, 16, 512, kSwizzle64);
+            }
+            mma_bf16(ts, da, db, id1, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar->s_full[jj & 1]);
+          if (k == n - 1) mma_commit(&bar->q_empty);
+          if (k >= 1 && !gemm2(jj - 1, k == 1)) ok = false;
+        }
+        if (!ok) break;
+        if (!gemm2(j + n - 1, n == 1)) break;
+        j += n;
+        ++p;
+      }
+      // drain: every MMA issued above has completed before TMEM / smem go away
+      mma_commit(&bar->drain);
+      mbar_wait_drain(&bar->drain, 0, lim);
+    }
+  } else {
+    // ------------------------------------------------------------ exchange, softmax, epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                 // query row within the tile = TMEM lane
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const bool row_valid = r < rows_valid;
+    const int qi = (row0 + r) / a.n_heads;             // query token of this row
+    const uint32_t x_peer = mapa(smem_u32(x_s), peer);
+    const uint32_t xfull_peer = mapa(smem_u32(&bar->x_full[0]), peer);
+    const int ltid = threadIdx.x - 64;                 // 0..127
+    // waits are warp-uniform: the TMEM loads and stores that follow are warp-collective
+    auto wwait = [&](uint64_t* b, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, status, lim));
+    };
+    PieceIter it(plan, a.batch, w);
+    Piece pc;
+    int j = 0;
+    bool ok = true;
+    while (ok && it.next(&pc)) {
+      const int n = pc.pg_end - pc.pg_begin;
+      const int len = a.seq_lens[pc.b];
+      const int vis_last = len - a.nq + qi;            // last key index this row may see
+      float m_used = -INFINITY, l = 0.f;
+      for (int k = 0; k < n; ++k) {
+        const int jj = j + k;
+        const int slot = jj & 1;
+        const int pg = pc.pg_begin + k;
+        if (!wwait(&bar->s_full[slot], (jj >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        float s[64];
+        tmem_ld32(tmem + kTmemS + 64 * slot + lane_off, s);
+        tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32, s + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->s_empty[slot]);
+
+        // this CTA's partial, in log2 units, rounded to fp16, to the peer
+        uint32_t h[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h[i] = pack_half2(s[2 * i] * prm.scale_log2, s[2 * i + 1] * prm.scale_log2);
+        if (jj >= 2 && !wwait(&bar->x_free[slot], ((jj >> 1) - 1) & 1)) { ok = false; break; }
+        const uint32_t dst = x_peer + slot * kXBytes + r * 128;
+        const uint32_t rbar = xfull_peer + slot * 8;
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8)
+          st_async_v4(dst + ((k8 ^ (r & 7)) << 4), make_uint4(h[4 * k8], h[4 * k8 + 1], h[4 * k8 + 2], h[4 * k8 + 3]),
+                      rbar);
+        if (ltid == 0) mbar_arrive_expect_tx(&bar->x_full[slot], kXBytes);
+        if (!wwait(&bar->x_full[slot], (jj >> 1) & 1)) { ok = false; break; }
+
+        // full scores S = fp16(S_own) + fp16(S_peer), masked
+        const int id = a.page_table[(size_t)pc.b * a.max_pages + pg];
+        const bool page_ok = id >= 0 && id < a.num_pages;
+        if (!page_ok && ltid == 0) record_status(status, MLA_ERR_RANGE);
+        const int base = pg * 64;
+        const int nvalid = page_ok ? min(64, len - base) : 0;
+        const int lim_key = row_valid ? min(nvalid - 1, vis_last - base) : -1;  // keys 0..lim_key visible
+        unsigned char* xrow = x_s + slot * kXBytes + r * 128;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xrow + ((k8 ^ (r & 7)) << 4));
+          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 o2 = unpack_half2(h[4 * k8 + e]);
+            const float2 p2 = unpack_half2(pv[e]);
+            const int i0 = 8 * k8 + 2 * e;
+            s[i0] = (i0 <= lim_key) ? o2.x + p2.x : -INFINITY;
+            s[i0 + 1] = (i0 + 1 <= lim_key) ? o2.y + p2.y : -INFINITY;
+            mx = fmaxf(mx, fmaxf(s[i0], s[i0 + 1]));
+          }
+        }
+        // lazy running max: rescale O and l only when the max grows by more than 2^8
+        const float m_new = fmaxf(m_used, mx);
+        const bool grow = m_new > m_used + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, grow && k > 0 && m_used != -INFINITY)) {
+          const float alpha = (grow && m_used != -INFINITY) ? ex2(m_used - m_new) : 1.f;
+          const int jp = jj - 1;  // O must hold every earlier page of this piece
+          if (!wwait(&bar->o_done[jp & 1], (jp >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < 256; cc += 32) {
+            float o[32];
+            tmem_ld32(tmem + lane_off + cc, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tmem + lane_off + cc, o);
+          }
+          tmem_wait_st();
+          l *= alpha;
+        }
+        if (grow) m_used = m_new;
+        const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
+        float psum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(s[2 * i] - m_ref), p1 = ex2(s[2 * i + 1] - m_ref);  // ex2(-inf) = 0
+          psum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        l += psum;
+        // P (bf16, 128-byte swizzled K-major rows) replaces the peer's scores in place
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8)
+          *reinterpret_cast<uint4*>(xrow + ((k8 ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * k8], pk[4 * k8 + 1], pk[4 * k8 + 2], pk[4 * k8 + 3]);
+        // cache slots past the sequence (or a page never loaded) feed the value
+        // product: zero their latent columns so that 0 * garbage cannot make NaN
+        if (nvalid < 64) {
+          unsigned char* pgb = pg_s + (jj % kStages) * kPageBytes;
+          const int nz = (64 - nvalid) * 4 * 8;          // 16-byte chunks to clear
+          for (int t = ltid; t < nz; t += 128) {
+            const int row = nvalid + t / 32, blk = (t / 8) & 3, ch = t & 7;
+            *reinterpret_cast<uint4*>(pgb + blk * 8192 + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();  // orders an O rescale (tcgen05.st) before the value MMA
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->p_full[slot]);
+      }
+      if (!ok) break;
+
+      // epilogue: O / l and lse of this piece
+      const int jl = j + n - 1;
+      if (!wwait(&bar->o_done[jl & 1], (jl >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const int grow_row = row0 + r;
+      float* dst = a.part_o + ((size_t)pc.id * prm.rows_total + grow_row) * a.d_c + c * 256;
+#pragma unroll 1
+      for (int cc = 0; cc < 256; cc += 32) {
+        float o[32];
+        tmem_ld32(tmem + lane_off + cc, o);
+        tmem_wait_ld();
+        if (row_valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + cc + i) =
+                make_float4(o[i] * inv_l, o[i + 1] * inv_l, o[i + 2] * inv_l, o[i + 3] * inv_l);
+        }
+      }
+      if (row_valid && c == 0)
+        a.part_lse[(size_t)pc.id * prm.rows_total + grow_row] =
+            l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->o_free);
+      j += n;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();  // the peer no longer stores into this CTA's shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over [rows, 576] with row stride 1152 bytes, box [box_rows, box_cols].
+bool encode_rows576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                    CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {576, rows};
+  cuuint64_t strides[1] = {576 * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool decode_tc_supported(int d_c, int d_rope, int page_size) { return d_c == 512 && d_rope == 64 && page_size == 64; }
+
+int decode_tc_workers(int sms, int rows_total) {
+  const int tiles = (rows_total + 127) / 128;
+  const int g = (sms / 2) / tiles;
+  return g < 1 ? 1 : g;
+}
+
+cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cudaStream_t stream) {
+  const int rows_total = a.nq * a.n_heads;
+  CUtensorMap tq128, tq64, tp128, tp64;
+  const uint64_t qrows = (uint64_t)a.batch * rows_total;
+  const uint64_t prows = (uint64_t)a.num_pages * 64;
+  if (!encode_rows576(&tq128, a.q_lat, qrows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows576(&tq64, a.q_lat, qrows, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_rows576(&tp128, a.pool, prows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_rows576(&tp64, a.pool, prows, 32, 64, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  TcParams prm;
+  prm.d = a;
+  prm.rows_total = rows_total;
+  prm.scale_log2 = a.scale * 1.4426950408889634f;
+  prm.spin_limit = spin_limit;
+  cudaError_t e = cudaFuncSetAttribute(decode_split_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.G, (rows_total + 127) / 128, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_split_tc_kernel, tq128, tq64, tp128, tp64, prm);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace mla
