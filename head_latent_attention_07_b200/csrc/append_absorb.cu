@@ -8,6 +8,7 @@
 // up to 16 tokens held on chip.
 #include "common.cuh"
 #include "decode.h"
+#include "mma_frag.cuh"
 
 namespace mla {
 
@@ -16,87 +17,188 @@ namespace {
 constexpr int kTokBlk = 16;
 
 // ------------------------------------------------------------------ append
-constexpr int kAppRows = 4;     // output rows (of d_c + d_rope) per CTA, one per warp
-constexpr int kAppK = 1024;     // hidden-state columns staged per step
+// [c || k^] rows = w_dkv [R x D] . h^T [D x T] on the tensor cores: one CTA per
+// 16-row tile of w_dkv and 16 tokens; its 8 warps split the reduction over D
+// in 32-wide slices (mma_frag.cuh), their partial tiles are summed in shared
+// memory, then RoPE is applied to the k^ rows and the bf16 row goes to its slot.
+constexpr int kAppWarps = 8;
+constexpr int kAppSplit = 4;   // CTAs of a cluster splitting the reduction over D
 
-__global__ void __launch_bounds__(kAppRows * 32)
+__global__ void __launch_bounds__(kAppWarps * 32)
 append_latent_kernel(AppendArgs a) {
-  __shared__ __align__(16) uint16_t h_s[kTokBlk * kAppK];
-  __shared__ float vals[kAppRows][kTokBlk];
+  __shared__ float part[kAppWarps][16][17];
+  __shared__ float red[kAppSplit][16][17];   // cluster leader: the split CTAs' tiles
   const int R = a.d_c + a.d_rope;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r0 = blockIdx.x * kAppRows;
+  const int g = lane >> 2, q = lane & 3;
+  const int m0 = blockIdx.x * 16;
   const int t0 = blockIdx.y * kTokBlk;
-  const int r = r0 + warp;
-  float acc[kTokBlk];
+  uint32_t split;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(split));
+  const int ra_row = m0 + g, rb_row = m0 + g + 8;
+  const int ta = t0 + g, tb = t0 + g + 8;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+  const int nslices = (a.d_model + 31) / 32;
+  // slices of this CTA's quarter, interleaved over its warps; 4 per batch of loads
+  for (int base = split * kAppWarps + warp; base < nslices; base += 4 * kAppWarps * kAppSplit) {
+    uint4 ra[4], rb[4], ha[4], hb[4];
 #pragma unroll
-  for (int j = 0; j < kTokBlk; ++j) acc[j] = 0.f;
-
-  for (int k0 = 0; k0 < a.d_model; k0 += kAppK) {
-    for (int idx = threadIdx.x; idx < kTokBlk * (kAppK / 8); idx += blockDim.x) {
-      const int j = idx / (kAppK / 8), v = idx % (kAppK / 8);
-      const int col = k0 + v * 8;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (t0 + j < a.n_tokens && col < a.d_model)
-        u = *reinterpret_cast<const uint4*>(a.h + (size_t)(t0 + j) * a.d_model + col);
-      reinterpret_cast<uint4*>(h_s)[idx] = u;
+    for (int u = 0; u < 4; ++u) {
+      const int sl = base + u * kAppWarps * kAppSplit;
+      const int kk = sl * 32 + 8 * q;
+      const bool kin = sl < nslices && kk < a.d_model;
+      ra[u] = (kin && ra_row < R) ? ldg_stream(a.w_dkv + (size_t)ra_row * a.d_model + kk) : z;
+      rb[u] = (kin && rb_row < R) ? ldg_stream(a.w_dkv + (size_t)rb_row * a.d_model + kk) : z;
+      ha[u] = (kin && ta < a.n_tokens) ? *reinterpret_cast<const uint4*>(a.h + (size_t)ta * a.d_model + kk) : z;
+      hb[u] = (kin && tb < a.n_tokens) ? *reinterpret_cast<const uint4*>(a.h + (size_t)tb * a.d_model + kk) : z;
     }
-    __syncthreads();
-    if (r < R) {
-      const uint16_t* wrow = a.w_dkv + (size_t)r * a.d_model + k0;
-      const int nv = min(kAppK, a.d_model - k0) / 8;
-      for (int v = lane; v < nv; v += 32) {
-        float wv[8];
-        unpack8(ldg_stream(wrow + v * 8), wv);
 #pragma unroll
-        for (int j = 0; j < kTokBlk; ++j) {
-          float hv[8];
-          unpack8(reinterpret_cast<const uint4*>(h_s + j * kAppK)[v], hv);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) acc[j] += wv[k] * hv[k];
-        }
-      }
+    for (int u = 0; u < 4; ++u) {
+      mma_k32(d0, ra[u], rb[u], ha[u]);
+      mma_k32(d1, ra[u], rb[u], hb[u]);
     }
-    __syncthreads();
   }
+  // fragment -> part[warp][row][token]
 #pragma unroll
-  for (int j = 0; j < kTokBlk; ++j) {
-    const float s = warp_sum(acc[j]);
-    if (lane == j) vals[warp][j] = s;
+  for (int e = 0; e < 4; ++e) {
+    const int row = g + ((e & 2) ? 8 : 0), tok = 2 * q + (e & 1);
+    part[warp][row][tok] = d0[e];
+    part[warp][row][tok + 8] = d1[e];
   }
   __syncthreads();
-
-  // store: thread (row rr, token j); RoPE rows pair up inside the CTA
-  // (r0 and d_c are multiples of kAppRows, hence even)
-  for (int idx = threadIdx.x; idx < kAppRows * kTokBlk; idx += blockDim.x) {
-    const int rr = idx / kTokBlk, j = idx % kTokBlk;
-    const int row = r0 + rr, t = t0 + j;
-    if (row >= R || t >= a.n_tokens) continue;
-    const int seq = a.seq_idx[t], p = a.pos[t];
-    if (seq < 0 || seq >= a.batch || p < 0 || p >= a.max_pages * a.page_size) {
-      record_status(a.dev_status, MLA_ERR_RANGE);
-      continue;
-    }
-    const int page = a.page_table[(size_t)seq * a.max_pages + p / a.page_size];
-    if (page < 0 || page >= a.num_pages) {
-      record_status(a.dev_status, MLA_ERR_RANGE);
-      continue;
-    }
-    float val = vals[rr][j];
-    if (row >= a.d_c) {
-      const int q = row - a.d_c;          // channel within the RoPE key
-      float c, s;
-      rope_cos_sin(p, q >> 1, a.d_rope, a.theta, &c, &s);
-      const float x0 = vals[rr & ~1][j], x1 = vals[rr | 1][j];
-      val = (q & 1) ? x0 * s + x1 * c : x0 * c - x1 * s;
-    }
-    a.pool[((size_t)page * a.page_size + p % a.page_size) * R + row] = f32_to_bf16(val);
+  {
+    // this CTA's tile -> slot `split` of the leader's shared memory
+    const int row = threadIdx.x >> 4, tok = threadIdx.x & 15;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAppWarps; ++w) v += part[w][row][tok];
+    const uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(&red[split][row][tok]));
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(local));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
   }
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (split != 0) return;
+  __shared__ float vals[16][17];
+  {
+    const int row = threadIdx.x >> 4, tok = threadIdx.x & 15;
+    vals[row][tok] = (red[0][row][tok] + red[1][row][tok]) + (red[2][row][tok] + red[3][row][tok]);
+  }
+  __syncthreads();
+  // store: thread (row, token); RoPE rows pair up inside the tile (m0 and d_c are even)
+  const int rr = threadIdx.x >> 4, j = threadIdx.x & 15;
+  const int row = m0 + rr, t = t0 + j;
+  if (row >= R || t >= a.n_tokens) return;
+  const int seq = a.seq_idx[t], p = a.pos[t];
+  if (seq < 0 || seq >= a.batch || p < 0 || p >= a.max_pages * a.page_size) {
+    record_status(a.dev_status, MLA_ERR_RANGE);
+    return;
+  }
+  const int page = a.page_table[(size_t)seq * a.max_pages + p / a.page_size];
+  if (page < 0 || page >= a.num_pages) {
+    record_status(a.dev_status, MLA_ERR_RANGE);
+    return;
+  }
+  float val = vals[rr][j];
+  if (row >= a.d_c) {
+    const int qch = row - a.d_c;          // channel within the RoPE key
+    float c, s;
+    rope_cos_sin(p, qch >> 1, a.d_rope, a.theta, &c, &s);
+    const float x0 = vals[rr & ~1][j], x1 = vals[rr | 1][j];
+    val = (qch & 1) ? x0 * s + x1 * c : x0 * c - x1 * s;
+  }
+  a.pool[((size_t)page * a.page_size + p % a.page_size) * R + row] = f32_to_bf16(val);
 }
 
 // ------------------------------------------------------------------ absorb
 constexpr int kAbsThreads = 256;
 
+// RoPE(q_rope, pos) of one head for up to kTokBlk tokens.
+__device__ __forceinline__ void absorb_rope_part(const AbsorbArgs& a, int h, int t0) {
+  const int dq = a.qk_nope + a.d_rope;
+  const int R = a.d_c + a.d_rope;
+  const int npair = a.d_rope / 2;
+  for (int idx = threadIdx.x; idx < kTokBlk * npair; idx += blockDim.x) {
+    const int k = idx / npair, i = idx % npair;
+    const int t = t0 + k;
+    if (t >= a.n_tokens) continue;
+    const uint16_t* src = a.q + ((size_t)t * a.n_heads + h) * dq + a.qk_nope + 2 * i;
+    const float x0 = bf16_to_f32(src[0]), x1 = bf16_to_f32(src[1]);
+    float c, s;
+    rope_cos_sin(a.pos[t], i, a.d_rope, a.theta, &c, &s);
+    *reinterpret_cast<uint32_t*>(a.q_lat + ((size_t)t * a.n_heads + h) * R + a.d_c + 2 * i) =
+        pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
+  }
+}
+
+// q~ = W_UK,h^T q_nope on the tensor cores, one CTA per (head, 16 tokens):
+// D^T [16 tokens x d_c] = Q [16 x qk_nope] . W_UK,h [qk_nope x d_c].  W_UK,h is
+// staged in shared memory (rows padded by 16 bytes) and read as B fragments with
+// ldmatrix.trans; each of the 8 warps owns d_c / 8 output columns.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__global__ void __launch_bounds__(kAbsThreads)
+absorb_q_mma_kernel(AbsorbArgs a) {
+  extern __shared__ __align__(16) uint16_t wsm[];   // [qk_nope][d_c + 8]
+  const int h = blockIdx.x;
+  const int t0 = blockIdx.y * kTokBlk;
+  const int dq = a.qk_nope + a.d_rope;
+  const int R = a.d_c + a.d_rope;
+  const int ws = a.d_c + 8;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, q4 = lane & 3;
+  // stage W_UK,h
+  const uint16_t* wh = a.w_uk + (size_t)h * a.qk_nope * a.d_c;
+  const int cpr = a.d_c / 8;                        // 16-byte chunks per row
+  for (int idx = threadIdx.x; idx < a.qk_nope * cpr; idx += blockDim.x) {  // all copies in flight at once
+    const int i = idx / cpr, cch = idx % cpr;
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(wsm + i * ws + cch * 8));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(wh + (size_t)i * a.d_c + cch * 8)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  absorb_rope_part(a, h, t0);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  const int ta = t0 + g, tb = t0 + g + 8;
+  const uint16_t* qa = a.q + ((size_t)ta * a.n_heads + h) * dq;
+  const uint16_t* qb = a.q + ((size_t)tb * a.n_heads + h) * dq;
+  const bool va = ta < a.n_tokens, vb = tb < a.n_tokens;
+  const int ntiles = a.d_c / 8;
+  for (int nt0 = warp * 2; nt0 < ntiles; nt0 += 16) {  // pairs of 8-column tiles
+    float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const int j0 = nt0 * 8;
+    for (int i0 = 0; i0 < a.qk_nope; i0 += 16) {
+      const int ia = i0 + 2 * q4;
+      const uint32_t a0 = va ? *reinterpret_cast<const uint32_t*>(qa + ia) : 0u;
+      const uint32_t a1 = vb ? *reinterpret_cast<const uint32_t*>(qb + ia) : 0u;
+      const uint32_t a2 = va ? *reinterpret_cast<const uint32_t*>(qa + ia + 8) : 0u;
+      const uint32_t a3 = vb ? *reinterpret_cast<const uint32_t*>(qb + ia + 8) : 0u;
+      // tiles: 0 = W[i0..+8][j0..+8], 1 = W[i0+8..][j0..], 2 = W[i0..][j0+8..], 3 = W[i0+8..][j0+8..]
+      const int tile = lane >> 3, rr = lane & 7;
+      const int wi = i0 + rr + ((tile & 1) ? 8 : 0);
+      const int wj = j0 + ((tile & 2) ? 8 : 0);
+      uint32_t b[4];
+      ldsm_x4_trans(static_cast<uint32_t>(__cvta_generic_to_shared(wsm + wi * ws + wj)), b);
+      mma_16816(d[0], a0, a1, a2, a3, b[0], b[1]);
+      if (nt0 + 1 < ntiles) mma_16816(d[1], a0, a1, a2, a3, b[2], b[3]);
+    }
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      const int j = j0 + 8 * n + 2 * q4;
+      if (nt0 + n >= ntiles) continue;
+      if (va) *reinterpret_cast<uint32_t*>(a.q_lat + ((size_t)ta * a.n_heads + h) * R + j) = pack_bf16x2(d[n][0], d[n][1]);
+      if (vb) *reinterpret_cast<uint32_t*>(a.q_lat + ((size_t)tb * a.n_heads + h) * R + j) = pack_bf16x2(d[n][2], d[n][3]);
+    }
+  }
+}
+
+// CUDA-core fallback for shapes whose W_UK,h does not fit in shared memory.
 __global__ void __launch_bounds__(kAbsThreads)
 absorb_q_kernel(AbsorbArgs a) {
   extern __shared__ __align__(16) float qn[];   // [kTokBlk][qk_nope]
@@ -134,37 +236,44 @@ absorb_q_kernel(AbsorbArgs a) {
             pack_bf16x2(acc0[k], acc1[k]);
     }
   }
-  // positional part: RoPE(q_rope, pos)
-  const int npair = a.d_rope / 2;
-  for (int idx = threadIdx.x; idx < kTokBlk * npair; idx += blockDim.x) {
-    const int k = idx / npair, i = idx % npair;
-    const int t = t0 + k;
-    if (t >= a.n_tokens) continue;
-    const uint16_t* src = a.q + ((size_t)t * a.n_heads + h) * dq + a.qk_nope + 2 * i;
-    const float x0 = bf16_to_f32(src[0]), x1 = bf16_to_f32(src[1]);
-    float c, s;
-    rope_cos_sin(a.pos[t], i, a.d_rope, a.theta, &c, &s);
-    *reinterpret_cast<uint32_t*>(a.q_lat + ((size_t)t * a.n_heads + h) * R + a.d_c + 2 * i) =
-        pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
-  }
+  absorb_rope_part(a, h, t0);
 }
 
 }  // namespace
 
 cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream) {
   const int R = a.d_c + a.d_rope;
-  dim3 grid((R + kAppRows - 1) / kAppRows, (a.n_tokens + kTokBlk - 1) / kTokBlk);
-  append_latent_kernel<<<grid, kAppRows * 32, 0, stream>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((R + 15) / 16, (a.n_tokens + kTokBlk - 1) / kTokBlk, kAppSplit);
+  cfg.blockDim = dim3(kAppWarps * 32, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = kAppSplit;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, append_latent_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream) {
+  dim3 grid(a.n_heads, (a.n_tokens + kTokBlk - 1) / kTokBlk);
+  const size_t wsmem = (size_t)a.qk_nope * (a.d_c + 8) * 2;
+  if (a.qk_nope % 16 == 0 && a.d_c % 8 == 0 && wsmem <= 200 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(absorb_q_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)wsmem);
+    if (e != cudaSuccess) return e;
+    absorb_q_mma_kernel<<<grid, kAbsThreads, wsmem, stream>>>(a);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)kTokBlk * a.qk_nope * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(absorb_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(a.n_heads, (a.n_tokens + kTokBlk - 1) / kTokBlk);
   absorb_q_kernel<<<grid, kAbsThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

@@ -36,12 +36,10 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
   f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
 }
 
-// Read-only global load that does not allocate in L1 (streamed once).
+// Global load of data read once (cache-streaming); the compiler may schedule
+// it freely, so several can be in flight per thread.
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-  return r;
+  return __ldcs(reinterpret_cast<const uint4*>(p));
 }
 
 // ---------------------------------------------------------------- RoPE

@@ -5,11 +5,15 @@
 //   o_lat = sum_s exp(lse_s - LSE) * O_s          (O_s already normalised per piece)
 //   out[t][h][v] = sum_c W_UV[h][v][c] * o_lat[c]  (values up-projected once, after
 //                                                   attending over latents)
-// One CTA = one head and up to kTok query tokens, so W_UV,h is streamed once per
-// group of kTok tokens and reused from registers across them.
+// One CTA = one head and up to 16 query tokens.  The merge runs on all 256
+// threads (coalesced reads of the partials); the up-projection is a
+// [v_head x d_c] x [d_c x 16] product on the tensor cores (mma.sync, fp32
+// accumulate) with o_lat split into two bf16 terms (hi + lo), which keeps about
+// 16 bits of its mantissa.  W_UV,h is streamed once per group of 16 tokens.
 #include "common.cuh"
-#include "plan.cuh"
 #include "decode.h"
+#include "mma_frag.cuh"
+#include "plan.cuh"
 
 namespace mla {
 
@@ -18,11 +22,16 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTok = 16;
 
+__device__ __forceinline__ uint4 ld_nc_v4(const uint16_t* p) { return ldg_stream(p); }
+
 __global__ void __launch_bounds__(kThreads)
 decode_combine_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PlanSmem* ps = reinterpret_cast<PlanSmem*>(smem_raw);
-  float* olat = reinterpret_cast<float*>(smem_raw + ((sizeof(PlanSmem) + 15) & ~size_t(15)));  // [kTok][d_c]
+  const int kpad = ((a.d_c + 31) & ~31);                 // reduction length padded to 32
+  const int ostride = kpad + 8;                          // bf16 row stride (16-byte pad: no bank conflicts)
+  uint16_t* o_hi = reinterpret_cast<uint16_t*>(smem_raw + ((sizeof(PlanSmem) + 15) & ~size_t(15)));
+  uint16_t* o_lo = o_hi + kTok * ostride;
 
   build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr);
   const int h = blockIdx.x;
@@ -31,77 +40,126 @@ decode_combine_kernel(DecodeArgs a) {
   const int rows_total = a.nq * a.n_heads;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // 1. merge: one warp per token
-  for (int j = warp; j < kTok; j += kThreads / 32) {
+  // 1. merge: 16 threads per token, each owning 8 consecutive columns per 128
+  {
+    const int j = tid >> 4, sub = tid & 15;
     const int t = t0 + j;
-    float* dst = olat + j * a.d_c;
-    if (t >= T) {
-      for (int c = lane; c < a.d_c; c += 32) dst[c] = 0.f;
-      continue;
-    }
-    const int b = t / a.nq, i = t % a.nq;
-    const int row = i * a.n_heads + h;
-    const int pb = ps->piece_begin[b], np = ps->piece_begin[b + 1] - pb;
-    float mx = -INFINITY;
-    for (int s = lane; s < np; s += 32) mx = fmaxf(mx, a.part_lse[(size_t)(pb + s) * rows_total + row]);
-    mx = warp_max(mx);
-    float tot = 0.f;
-    for (int s = lane; s < np; s += 32) {
-      const float l = a.part_lse[(size_t)(pb + s) * rows_total + row];
-      tot += (l == -INFINITY) ? 0.f : expf(l - mx);
-    }
-    tot = warp_sum(tot);
-    const bool empty = (mx == -INFINITY);
-    const float lse_all = empty ? -INFINITY : mx + logf(tot);
-    for (int c = lane * 4; c < a.d_c; c += 128) {
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (!empty) {
+    float lse_all = -INFINITY;
+    int pb = 0, np = 0, row = 0;
+    if (t < T) {
+      const int b = t / a.nq, i = t % a.nq;
+      row = i * a.n_heads + h;
+      pb = ps->piece_begin[b];
+      np = ps->piece_begin[b + 1] - pb;
+      float mx = -INFINITY;
+      for (int s = 0; s < np; ++s) mx = fmaxf(mx, a.part_lse[(size_t)(pb + s) * rows_total + row]);
+      if (mx != -INFINITY) {
+        float tot = 0.f;
         for (int s = 0; s < np; ++s) {
           const float l = a.part_lse[(size_t)(pb + s) * rows_total + row];
-          if (l == -INFINITY) continue;
-          const float wgt = expf(l - lse_all);
-          const float4 v = *reinterpret_cast<const float4*>(
-              a.part_o + ((size_t)(pb + s) * rows_total + row) * a.d_c + c);
-          o.x += wgt * v.x; o.y += wgt * v.y; o.z += wgt * v.z; o.w += wgt * v.w;
+          tot += (l == -INFINITY) ? 0.f : expf(l - mx);
+        }
+        lse_all = mx + logf(tot);
+      }
+      if (sub == 0 && a.lse != nullptr) a.lse[(size_t)t * a.n_heads + h] = lse_all;
+    }
+    for (int c0 = sub * 8; c0 < kpad; c0 += 128) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+      if (lse_all != -INFINITY && c0 < a.d_c) {
+        for (int s0 = 0; s0 < np; s0 += 4) {         // four pieces' loads in flight at once
+          float4 v0[4], v1[4];
+          float wgt[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int s = s0 + u;
+            wgt[u] = 0.f;
+            v0[u] = v1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s < np) {
+              const float l = a.part_lse[(size_t)(pb + s) * rows_total + row];
+              const float* src = a.part_o + ((size_t)(pb + s) * rows_total + row) * a.d_c + c0;
+              v0[u] = *reinterpret_cast<const float4*>(src);
+              v1[u] = *reinterpret_cast<const float4*>(src + 4);
+              wgt[u] = (l == -INFINITY) ? 0.f : expf(l - lse_all);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            acc[0] += wgt[u] * v0[u].x; acc[1] += wgt[u] * v0[u].y;
+            acc[2] += wgt[u] * v0[u].z; acc[3] += wgt[u] * v0[u].w;
+            acc[4] += wgt[u] * v1[u].x; acc[5] += wgt[u] * v1[u].y;
+            acc[6] += wgt[u] * v1[u].z; acc[7] += wgt[u] * v1[u].w;
+          }
         }
       }
-      *reinterpret_cast<float4*>(dst + c) = o;
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = acc[2 * e], x1 = acc[2 * e + 1];
+        hi[e] = pack_bf16x2(x0, x1);
+        lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+      }
+      *reinterpret_cast<uint4*>(o_hi + j * ostride + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(o_lo + j * ostride + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    if (lane == 0 && a.lse != nullptr) a.lse[(size_t)t * a.n_heads + h] = lse_all;
   }
   __syncthreads();
 
-  // 2. out[t][h][v] = W_UV,h[v] . o_lat[t]: warp per value row, lanes split d_c
-  const int cvec = a.d_c / 8;
+  // 2. out[t][v] = sum_c W_UV,h[v][c] o_lat[t][c]: warp per 16 value rows,
+  //    two 8-token tiles, reduction in 32-wide slices (see mma_frag.cuh)
+  const int g = lane >> 2, q = lane & 3;
   const uint16_t* wh = a.w_uv + (size_t)h * a.v_head * a.d_c;
-  for (int v = warp; v < a.v_head; v += kThreads / 32) {
-    float part[kTok];
+  for (int m0 = warp * 16; m0 < a.v_head; m0 += 8 * 16) {
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int va = m0 + g, vb = m0 + g + 8;
+    for (int kb = 0; kb < kpad; kb += 128) {          // four 32-wide slices' weights in flight at once
+      uint4 ra[4], rb[4];
+      const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int j = 0; j < kTok; ++j) part[j] = 0.f;
-    for (int k = lane; k < cvec; k += 32) {
-      float wv[8];
-      unpack8(ldg_stream(wh + (size_t)v * a.d_c + k * 8), wv);
+      for (int u = 0; u < 4; ++u) {
+        const int kk = kb + 32 * u + 8 * q;
+        const bool kin = kk < a.d_c;
+        ra[u] = (kin && va < a.v_head) ? ld_nc_v4(wh + (size_t)va * a.d_c + kk) : z;
+        rb[u] = (kin && vb < a.v_head) ? ld_nc_v4(wh + (size_t)vb * a.d_c + kk) : z;
+      }
 #pragma unroll
-      for (int j = 0; j < kTok; ++j) {
-        const float4 o0 = *reinterpret_cast<const float4*>(olat + j * a.d_c + k * 8);
-        const float4 o1 = *reinterpret_cast<const float4*>(olat + j * a.d_c + k * 8 + 4);
-        part[j] += wv[0] * o0.x + wv[1] * o0.y + wv[2] * o0.z + wv[3] * o0.w +
-                   wv[4] * o1.x + wv[5] * o1.y + wv[6] * o1.z + wv[7] * o1.w;
+      for (int u = 0; u < 4; ++u) {
+        const int kk = kb + 32 * u + 8 * q;
+        if (kk >= kpad) break;
+        const uint4 h0 = *reinterpret_cast<const uint4*>(o_hi + g * ostride + kk);
+        const uint4 l0 = *reinterpret_cast<const uint4*>(o_lo + g * ostride + kk);
+        const uint4 h1 = *reinterpret_cast<const uint4*>(o_hi + (g + 8) * ostride + kk);
+        const uint4 l1 = *reinterpret_cast<const uint4*>(o_lo + (g + 8) * ostride + kk);
+        mma_k32(d0, ra[u], rb[u], h0);
+        mma_k32(d0, ra[u], rb[u], l0);
+        mma_k32(d1, ra[u], rb[u], h1);
+        mma_k32(d1, ra[u], rb[u], l1);
       }
     }
+    // D fragment: (row g | g+8, token column 2q | 2q+1) of each 8-token tile
+    const float* dd[2] = {d0, d1};
 #pragma unroll
-    for (int j = 0; j < kTok; ++j) {
-      const float sum = warp_sum(part[j]);
-      const int t = t0 + j;
-      if (lane == j && t < T) a.out[((size_t)t * a.n_heads + h) * a.v_head + v] = f32_to_bf16(sum);
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int v = m0 + g + ((e & 2) ? 8 : 0);
+        const int t = t0 + nt * 8 + 2 * q + (e & 1);
+        if (v < a.v_head && t < T) a.out[((size_t)t * a.n_heads + h) * a.v_head + v] = f32_to_bf16(dd[nt][e]);
+      }
     }
   }
 }
 
 }  // namespace
 
+size_t decode_combine_smem_bytes(int d_c) {
+  const int kpad = ((d_c + 31) & ~31);
+  return ((sizeof(PlanSmem) + 15) & ~size_t(15)) + 2ull * kTok * (kpad + 8) * 2;
+}
+
 cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
-  const size_t smem = ((sizeof(PlanSmem) + 15) & ~size_t(15)) + (size_t)kTok * a.d_c * 4;
+  const size_t smem = decode_combine_smem_bytes(a.d_c);
   cudaError_t e = cudaFuncSetAttribute(decode_combine_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -9,18 +9,22 @@
 // pair, half by each CTA.  Per page (64 tokens):
 //   GEMM1   S_c[128 x 64]  = Q_c[128 x 288] . K_c[64 x 288]^T        (tcgen05, TMEM)
 //   swap    each CTA scales S_c to log2 units, rounds it to fp16 and stores it
-//           into its peer's shared memory (st.async); both CTAs then hold the same
-//           S = fp16(S_0) + fp16(S_1), the full 576-wide score (content + RoPE)
+//           into its peer's shared memory (st.async); each CTA then forms the
+//           full 576-wide score (content + RoPE) S = S_own + fp16(S_peer)
 //   softmax one thread per query row: running max / sum over the page, P in bf16
 //   GEMM2   O_c[128 x 256] += P[128 x 64] . C_c[64 x 256]               (tcgen05, TMEM)
-// Both CTAs compute the same softmax, so the two O halves share one normaliser.
 // The running max is only moved (and O rescaled in TMEM) when it grows by more
 // than 2^8; otherwise P is taken relative to the stale max (P <= 256).
 // TMEM: O_c uses columns [0, 256), the two S buffers [256, 320) and [320, 384).
 //
-// Warp roles (192 threads): warp 0 lane 0 issues TMA loads (query tile once per
-// piece, pages into a 3-stage ring), warp 1 owns TMEM and lane 0 issues the MMAs,
-// warps 2..5 (one per TMEM lane quarter) run the exchange, softmax and epilogue.
+// Warp roles (448 threads): warp 0 lane 0 issues TMA loads (query tile once per
+// piece, pages into a 3-stage ring, L2 prefetch further ahead), warp 1 owns TMEM
+// and lane 0 issues the MMAs (score GEMM up to two pages ahead of the value
+// GEMM), warps 2..5 (one per TMEM lane quarter) send this CTA's partial scores to
+// the peer, and warps 6..9 (one per lane quarter, one query row per thread) run
+// the softmax and epilogue.  Each CTA adds its own fp32 partial scores to the
+// peer's fp16 ones; the two CTAs' scores differ only by that rounding, and each
+// normalises its own half of O with its own running sum.
 // Every mbarrier wait is bounded: on time-out the kernel records MLA_ERR_TIMEOUT,
 // stops its loops, drains its own copies and MMAs and frees TMEM.
 #include <cuda.h>
@@ -39,8 +43,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, 4 exchange warps, 4 softmax warps
 constexpr int kStages = 3;
+constexpr int kPrefetch = 4;  // pages beyond the shared-memory ring prefetched into L2
 constexpr int kQBytes = 4 * 16384 + 8192;     // 4 latent blocks [128 x 64] + RoPE block [128 x 32]
 constexpr int kPageBytes = 4 * 8192 + 4096;   // 4 latent blocks [64 x 64]  + RoPE block [64 x 32]
 constexpr int kXBytes = 128 * 128;            // [128 rows x 64] fp16 scores, then bf16 P
@@ -50,10 +55,12 @@ constexpr int kOffX = kOffPg + kStages * kPageBytes;
 constexpr int kOffPlan = kOffX + 2 * kXBytes;
 constexpr int kOffBar = kOffPlan + ((int(sizeof(PlanSmem)) + 127) & ~127);
 constexpr int kNumBars = 24;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 64 + 1024;  // + misc + 1 KB alignment slack
+constexpr int kOffMisc = kOffBar + kNumBars * 8;       // TMEM base, abort flag, page metadata
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;       // + 1 KB alignment slack
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: rescale when the max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 256;              // first S buffer column
+constexpr uint32_t kTmemS = 256;              // S buffers: columns [256, 320) and [320, 384)
+constexpr uint32_t kTmemP = 384;              // P buffers (bf16 pairs): [384, 416) and [416, 448)
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffPg % 1024 == 0 && kPageBytes % 1024 == 0 && kOffX % 1024 == 0, "swizzle alignment");
@@ -105,6 +112,33 @@ struct PieceIter {
   }
 };
 
+// Walks the pages of worker w: jj counts pages across pieces, p counts pieces.
+struct PageCursor {
+  PieceIter it;
+  Piece pc;
+  int pg = 0, jj = -1, p = -1;
+  bool in_piece = false;
+  __device__ PageCursor(const PlanSmem* ps, int batch, int w) : it(ps, batch, w) {}
+  __device__ bool next() {
+    if (in_piece && pg + 1 < pc.pg_end) {
+      ++pg;
+      ++jj;
+      return true;
+    }
+    if (!it.next(&pc)) {
+      in_piece = false;
+      return false;
+    }
+    in_piece = true;
+    pg = pc.pg_begin;
+    ++jj;
+    ++p;
+    return true;
+  }
+  __device__ bool first() const { return pg == pc.pg_begin; }
+  __device__ bool last() const { return pg == pc.pg_end - 1; }
+};
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -112,6 +146,21 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
   return __half22float2(*reinterpret_cast<__half2*>(&v));
 }
+__device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// fp16 pair -> two fp32 values scaled by 2^-112 (exact for normal and zero
+// halves, sign kept), on the integer pipe: f = bits(x_fp16) re-based as fp32.
+// Multiplying by 2^112 restores the value.
+__device__ __forceinline__ float h_lo_scaled(uint32_t v) {
+  return __uint_as_float(((v & 0x8000u) << 16) | ((v & 0x7FFFu) << 13));
+}
+__device__ __forceinline__ float h_hi_scaled(uint32_t v) {
+  return __uint_as_float((v & 0x80000000u) | ((v >> 3) & 0x0FFFE000u));
+}
+constexpr float kTwo112 = 5.192296858534828e33f;  // 2^112
 
 __global__ void __launch_bounds__(kThreads, 1)
 decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_constant__ CUtensorMap tq64,
@@ -125,8 +174,9 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
   unsigned char* x_s = sm + kOffX;
   PlanSmem* plan = reinterpret_cast<PlanSmem*>(sm + kOffPlan);
   Bars* bar = reinterpret_cast<Bars*>(sm + kOffBar);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + kOffBar + kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffBar + kNumBars * 8 + 16);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 16);
+  int* stage_nvalid = reinterpret_cast<int*>(sm + kOffMisc + 32);   // [kStages] valid keys of the page
 
   const DecodeArgs& a = prm.d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -144,9 +194,9 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
     for (int s = 0; s < kStages; ++s) { mbar_init(&bar->pg_full[s], 1); mbar_init(&bar->pg_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->s_empty[s], 4);
+      mbar_init(&bar->s_empty[s], 8);   // 4 exchange warps + 4 softmax warps read S
       mbar_init(&bar->x_full[s], 1);
-      mbar_init(&bar->x_free[s], 1);
+      mbar_init(&bar->x_free[s], 1);   // the peer's value MMA of the page ran: its slot was read
       mbar_init(&bar->p_full[s], 4);
       mbar_init(&bar->o_done[s], 1);
     }
@@ -172,34 +222,55 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      PieceIter it(plan, a.batch, w);
-      Piece pc;
-      int j = 0, p = 0;
+      PageCursor cu(plan, a.batch, w);
+      // L2 prefetch runs kStages + kPrefetch pages ahead of the shared-memory loads;
+      // this CTA prefetches its 32 of the page's 64 rows (36 KB contiguous)
+      PageCursor pf(plan, a.batch, w);
+      bool more_pf = pf.next();
+      auto prefetch_next = [&]() {
+        if (!more_pf) return;
+        const int id = a.page_table[(size_t)pf.pc.b * a.max_pages + pf.pg];
+        if (id >= 0 && id < a.num_pages)
+          prefetch_l2(a.pool + ((size_t)id * 64 + 32 * c) * 576, 32 * 576 * 2);
+        more_pf = pf.next();
+      };
+      for (int i = 0; i < kStages + kPrefetch; ++i) prefetch_next();
       int issued[kStages] = {0, 0, 0}, issued_q = 0;
-      while (!*abort_flag && it.next(&pc)) {
-        if (p > 0 && !mbar_wait(&bar->q_empty, (p - 1) & 1, abort_flag, status, lim)) break;
-        ++issued_q;
-        const int qrow = pc.b * prm.rows_total + row0;
-        mbar_arrive_expect_tx(&bar->q_full, kQBytes);
-        for (int i = 0; i < 4; ++i) tma_load_2d(q_s + i * 16384, &tq128, c * 256 + 64 * i, qrow, &bar->q_full);
-        tma_load_2d(q_s + 65536, &tq64, 512 + 32 * c, qrow, &bar->q_full);
-        bool ok = true;
-        for (int pg = pc.pg_begin; pg < pc.pg_end; ++pg, ++j) {
-          const int st = j % kStages;
-          if (j >= kStages && !mbar_wait(&bar->pg_empty[st], ((j / kStages) - 1) & 1, abort_flag, status, lim)) {
-            ok = false;
-            break;
-          }
-          int id = a.page_table[(size_t)pc.b * a.max_pages + pg];
-          if (id < 0 || id >= a.num_pages) id = 0;  // never read: the softmax masks and zeroes it
-          unsigned char* dst = pg_s + st * kPageBytes;
-          mbar_arrive_expect_tx(&bar->pg_full[st], kPageBytes);
-          for (int i = 0; i < 4; ++i) tma_load_2d(dst + i * 8192, &tp128, c * 256 + 64 * i, id * 64, &bar->pg_full[st]);
-          tma_load_2d(dst + 32768, &tp64, 512 + 32 * c, id * 64, &bar->pg_full[st]);
-          ++issued[st];
+      bool more = cu.next();
+      int id_next = more ? a.page_table[(size_t)cu.pc.b * a.max_pages + cu.pg] : 0;
+      int len_next = more ? a.seq_lens[cu.pc.b] : 0;
+      while (more && !*abort_flag) {
+        const int jj = cu.jj;
+        int id = id_next;
+        const int nvalid_raw = min(64, len_next - cu.pg * 64);
+        if (cu.first()) {
+          if (cu.p > 0 && !mbar_wait(&bar->q_empty, (cu.p - 1) & 1, abort_flag, status, lim)) break;
+          const int qrow = cu.pc.b * prm.rows_total + row0;
+          mbar_arrive_expect_tx(&bar->q_full, kQBytes);
+          for (int i = 0; i < 4; ++i) tma_load_2d(q_s + i * 16384, &tq128, c * 256 + 64 * i, qrow, &bar->q_full);
+          tma_load_2d(q_s + 65536, &tq64, 512 + 32 * c, qrow, &bar->q_full);
+          ++issued_q;
         }
-        if (!ok) break;
-        ++p;
+        const int st = jj % kStages;
+        more = cu.next();
+        // the next page id is read while this stage drains
+        if (more) {
+          id_next = a.page_table[(size_t)cu.pc.b * a.max_pages + cu.pg];
+          len_next = a.seq_lens[cu.pc.b];
+        }
+        if (jj >= kStages && !mbar_wait(&bar->pg_empty[st], ((jj / kStages) - 1) & 1, abort_flag, status, lim)) break;
+        const bool page_ok = id >= 0 && id < a.num_pages;
+        if (!page_ok) {
+          record_status(status, MLA_ERR_RANGE);
+          id = 0;  // loaded but never used: all its keys are masked and its rows zeroed
+        }
+        stage_nvalid[st] = page_ok ? nvalid_raw : 0;  // published by the arrive below
+        unsigned char* dst = pg_s + st * kPageBytes;
+        mbar_arrive_expect_tx(&bar->pg_full[st], kPageBytes);
+        for (int i = 0; i < 4; ++i) tma_load_2d(dst + i * 8192, &tp128, c * 256 + 64 * i, id * 64, &bar->pg_full[st]);
+        tma_load_2d(dst + 32768, &tp64, 512 + 32 * c, id * 64, &bar->pg_full[st]);
+        ++issued[st];
+        prefetch_next();
       }
       if (*abort_flag) {
         // copies still in flight must land before this CTA's shared memory is released
@@ -210,223 +281,279 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Two in-order queues: GEMM1 (scores, up to two pages ahead) and GEMM2
+    // (values); each is issued as soon as its own inputs are ready.
     if (lane == 0) {
       const uint32_t id1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id2 = idesc_bf16_f32(128, 256, 0, 1);
-      PieceIter it(plan, a.batch, w);
-      Piece pc;
-      int j = 0, p = 0;
-      bool ok = true;
-      auto gemm2 = [&](int jj, bool first) -> bool {
-        if (first && p > 0 && !mbar_wait(&bar->o_free, (p - 1) & 1, abort_flag, status, lim)) return false;
-        if (!mbar_wait(&bar->p_full[jj & 1], (jj >> 1) & 1, abort_flag, status, lim)) return false;
-        tc_fence_after();
-        const uint32_t xa = smem_u32(x_s + (jj & 1) * kXBytes);
-        const uint32_t pb = smem_u32(pg_s + (jj % kStages) * kPageBytes);
+      const uint32_t qa = smem_u32(q_s);
+      PageCursor g1(plan, a.batch, w), g2(plan, a.batch, w);
+      bool has1 = g1.next(), has2 = g2.next();
+      bool q_ok = false;  // query tile of g1's piece is resident
+      long long t_last = clock64();
+      while (has1 || has2) {
+        bool progressed = false;
+        if (has2 && g2.jj < (has1 ? g1.jj : 0x7fffffff)) {
+          const int jj = g2.jj;
+          const bool first = g2.first();
+          const bool ready = (!(first && g2.p > 0) || mbar_test(&bar->o_free, (g2.p - 1) & 1)) &&
+                             mbar_test(&bar->p_full[jj & 1], (jj >> 1) & 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t pa = tmem + kTmemP + 32 * (jj & 1);
+            const uint32_t pb = smem_u32(pg_s + (jj % kStages) * kPageBytes);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t da = smem_desc(xa + ks * 32, 16, 1024, kSwizzle128);
-          const uint64_t db = smem_desc(pb + ks * 2048, 8192, 1024, kSwizzle128);
-          mma_bf16(tmem, da, db, id2, (first && ks == 0) ? 0u : 1u);
-        }
-        mma_commit(&bar->pg_empty[jj % kStages]);
-        mma_commit(&bar->o_done[jj & 1]);
-        mma_commit_mc(&bar->x_free[jj & 1], uint16_t(1u << peer));
-        return true;
-      };
-      while (ok && it.next(&pc)) {
-        const int n = pc.pg_end - pc.pg_begin;
-        if (!mbar_wait(&bar->q_full, p & 1, abort_flag, status, lim)) break;
-        const uint32_t qa = smem_u32(q_s);
-        for (int k = 0; k < n && ok; ++k) {
-          const int jj = j + k;
-          const int st = jj % kStages;
-          if (!mbar_wait(&bar->pg_full[st], (jj / kStages) & 1, abort_flag, status, lim) ||
-              (jj >= 2 && !mbar_wait(&bar->s_empty[jj & 1], ((jj >> 1) - 1) & 1, abort_flag, status, lim))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t pb = smem_u32(pg_s + st * kPageBytes);
-          const uint32_t ts = tmem + kTmemS + 64 * (jj & 1);
-#pragma unroll
-          for (int ks = 0; ks < 18; ++ks) {
-            uint64_t da, db;
-            if (ks < 16) {
-              da = smem_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128);
-              db = smem_desc(pb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128);
-            } else {
-              da = smem_desc(qa + 65536 + (ks - 16) * 32, 16, 512, kSwizzle64);
-              db = smem_desc(pb + 32768 + (ks - 16) * 32, 16, 512, kSwizzle64);
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t db = smem_desc(pb + ks * 2048, 8192, 1024, kSwizzle128);
+              mma_bf16_ts(tmem, pa + 8 * ks, db, id2, (first && ks == 0) ? 0u : 1u);
             }
-            mma_bf16(ts, da, db, id1, ks > 0 ? 1u : 0u);
+            mma_commit(&bar->pg_empty[jj % kStages]);
+            mma_commit(&bar->o_done[jj & 1]);
+            // this CTA's receive slot (jj & 1) has been read: the peer may send page jj + 2
+            mma_commit_mc(&bar->x_free[jj & 1], uint16_t(1u << peer));
+            has2 = g2.next();
+            progressed = true;
           }
-          mma_commit(&bar->s_full[jj & 1]);
-          if (k == n - 1) mma_commit(&bar->q_empty);
-          if (k >= 1 && !gemm2(jj - 1, k == 1)) ok = false;
         }
-        if (!ok) break;
-        if (!gemm2(j + n - 1, n == 1)) break;
-        j += n;
-        ++p;
+        // GEMM1(j) waits for GEMM2(j - 2) to be issued: the tensor pipe runs in
+        // order, and the value product gates more of the pipeline than the scores
+        if (has1 && (!has2 || g1.jj < g2.jj + 2)) {
+          const int jj = g1.jj;
+          const int st = jj % kStages;
+          if (g1.first() && !q_ok) q_ok = mbar_test(&bar->q_full, g1.p & 1);
+          const bool ready = (!g1.first() || q_ok) &&
+                             (jj < 2 || mbar_test(&bar->s_empty[jj & 1], ((jj >> 1) - 1) & 1)) &&
+                             mbar_test(&bar->pg_full[st], (jj / kStages) & 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t pb = smem_u32(pg_s + st * kPageBytes);
+            const uint32_t ts = tmem + kTmemS + 64 * (jj & 1);
+#pragma unroll
+            for (int ks = 0; ks < 18; ++ks) {
+              uint64_t da, db;
+              if (ks < 16) {
+                da = smem_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128);
+                db = smem_desc(pb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128);
+              } else {
+                da = smem_desc(qa + 65536 + (ks - 16) * 32, 16, 512, kSwizzle64);
+                db = smem_desc(pb + 32768 + (ks - 16) * 32, 16, 512, kSwizzle64);
+              }
+              mma_bf16(ts, da, db, id1, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar->s_full[jj & 1]);
+            if (g1.last()) {
+              mma_commit(&bar->q_empty);
+              q_ok = false;
+            }
+            has1 = g1.next();
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_last = clock64();
+        } else if (*abort_flag) {
+          break;
+        } else if (clock64() - t_last > lim) {
+          record_status(status, MLA_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
       }
       // drain: every MMA issued above has completed before TMEM / smem go away
       mma_commit(&bar->drain);
       mbar_wait_drain(&bar->drain, 0, lim);
     }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ exchange warps
+    // A(k): this CTA's partial scores S(k) out of TMEM, scaled to log2 units,
+    // rounded to fp16 and stored into the peer's receive slot (k & 1).  Runs up
+    // to two pages ahead of the softmax warps.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const uint32_t x_peer = mapa(smem_u32(x_s), peer);
+    const uint32_t xfull_peer = mapa(smem_u32(&bar->x_full[0]), peer);
+    auto wwait = [&](uint64_t* b, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, status, lim));
+    };
+    PageCursor ca(plan, a.batch, w);
+    while (ca.next()) {
+      const int jj = ca.jj;
+      const int slot = jj & 1;
+      if (!wwait(&bar->s_full[slot], (jj >> 1) & 1)) break;
+      tc_fence_after();
+      float sv[64];
+      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off, sv);
+      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32, sv + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->s_empty[slot]);
+      uint32_t h[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h[i] = pack_half2(sv[2 * i] * prm.scale_log2, sv[2 * i + 1] * prm.scale_log2);
+      // the peer's receive slot is free once its softmax warps have read page jj - 2
+      if (jj >= 2 && !wwait(&bar->x_free[slot], ((jj >> 1) - 1) & 1)) break;
+      const uint32_t dst = x_peer + slot * kXBytes + r * 128;
+      const uint32_t rbar = xfull_peer + slot * 8;
+#pragma unroll
+      for (int k8 = 0; k8 < 8; ++k8)
+        st_async_v4(dst + ((k8 ^ (r & 7)) << 4), make_uint4(h[4 * k8], h[4 * k8 + 1], h[4 * k8 + 2], h[4 * k8 + 3]),
+                    rbar);
+      if (warp == 2 && lane == 0) mbar_arrive_expect_tx(&bar->x_full[slot], kXBytes);
+    }
   } else {
-    // ------------------------------------------------------------ exchange, softmax, epilogue
+    // ------------------------------------------------------------ softmax warps
+    // B(k), one query row per thread, all 64 keys of the page:
+    //   S = own + peer: this CTA's fp32 partial (scaled) plus the peer's fp16 one,
+    //   masked online softmax, P(k) (bf16) into TMEM, O rescale when the max grew,
+    //   epilogue (O / l, lse) at the end of each piece.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // query row within the tile = TMEM lane
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const bool row_valid = r < rows_valid;
     const int qi = (row0 + r) / a.n_heads;             // query token of this row
-    const uint32_t x_peer = mapa(smem_u32(x_s), peer);
-    const uint32_t xfull_peer = mapa(smem_u32(&bar->x_full[0]), peer);
-    const int ltid = threadIdx.x - 64;                 // 0..127
-    // waits are warp-uniform: the TMEM loads and stores that follow are warp-collective
+    const int ltid = threadIdx.x - 192;                // 0..127
+    const float own_scale = prm.scale_log2 * (1.0f / kTwo112);  // own partial in the peer's 2^-112 units
     auto wwait = [&](uint64_t* b, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, status, lim));
     };
-    PieceIter it(plan, a.batch, w);
-    Piece pc;
-    int j = 0;
+
+    PageCursor cb(plan, a.batch, w);
+    float m_used = -INFINITY, l = 0.f;
+    int vis_last = 0;
     bool ok = true;
-    while (ok && it.next(&pc)) {
-      const int n = pc.pg_end - pc.pg_begin;
-      const int len = a.seq_lens[pc.b];
-      const int vis_last = len - a.nq + qi;            // last key index this row may see
-      float m_used = -INFINITY, l = 0.f;
-      for (int k = 0; k < n; ++k) {
-        const int jj = j + k;
-        const int slot = jj & 1;
-        const int pg = pc.pg_begin + k;
-        if (!wwait(&bar->s_full[slot], (jj >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        float s[64];
-        tmem_ld32(tmem + kTmemS + 64 * slot + lane_off, s);
-        tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32, s + 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->s_empty[slot]);
-
-        // this CTA's partial, in log2 units, rounded to fp16, to the peer
-        uint32_t h[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) h[i] = pack_half2(s[2 * i] * prm.scale_log2, s[2 * i + 1] * prm.scale_log2);
-        if (jj >= 2 && !wwait(&bar->x_free[slot], ((jj >> 1) - 1) & 1)) { ok = false; break; }
-        const uint32_t dst = x_peer + slot * kXBytes + r * 128;
-        const uint32_t rbar = xfull_peer + slot * 8;
-#pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8)
-          st_async_v4(dst + ((k8 ^ (r & 7)) << 4), make_uint4(h[4 * k8], h[4 * k8 + 1], h[4 * k8 + 2], h[4 * k8 + 3]),
-                      rbar);
-        if (ltid == 0) mbar_arrive_expect_tx(&bar->x_full[slot], kXBytes);
-        if (!wwait(&bar->x_full[slot], (jj >> 1) & 1)) { ok = false; break; }
-
-        // full scores S = fp16(S_own) + fp16(S_peer), masked
-        const int id = a.page_table[(size_t)pc.b * a.max_pages + pg];
-        const bool page_ok = id >= 0 && id < a.num_pages;
-        if (!page_ok && ltid == 0) record_status(status, MLA_ERR_RANGE);
-        const int base = pg * 64;
-        const int nvalid = page_ok ? min(64, len - base) : 0;
-        const int lim_key = row_valid ? min(nvalid - 1, vis_last - base) : -1;  // keys 0..lim_key visible
-        unsigned char* xrow = x_s + slot * kXBytes + r * 128;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xrow + ((k8 ^ (r & 7)) << 4));
-          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 o2 = unpack_half2(h[4 * k8 + e]);
-            const float2 p2 = unpack_half2(pv[e]);
-            const int i0 = 8 * k8 + 2 * e;
-            s[i0] = (i0 <= lim_key) ? o2.x + p2.x : -INFINITY;
-            s[i0 + 1] = (i0 + 1 <= lim_key) ? o2.y + p2.y : -INFINITY;
-            mx = fmaxf(mx, fmaxf(s[i0], s[i0 + 1]));
-          }
-        }
-        // lazy running max: rescale O and l only when the max grows by more than 2^8
-        const float m_new = fmaxf(m_used, mx);
-        const bool grow = m_new > m_used + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, grow && k > 0 && m_used != -INFINITY)) {
-          const float alpha = (grow && m_used != -INFINITY) ? ex2(m_used - m_new) : 1.f;
-          const int jp = jj - 1;  // O must hold every earlier page of this piece
-          if (!wwait(&bar->o_done[jp & 1], (jp >> 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int cc = 0; cc < 256; cc += 32) {
-            float o[32];
-            tmem_ld32(tmem + lane_off + cc, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tmem + lane_off + cc, o);
-          }
-          tmem_wait_st();
-          l *= alpha;
-        }
-        if (grow) m_used = m_new;
-        const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-        float psum = 0.f;
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(s[2 * i] - m_ref), p1 = ex2(s[2 * i + 1] - m_ref);  // ex2(-inf) = 0
-          psum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        l += psum;
-        // P (bf16, 128-byte swizzled K-major rows) replaces the peer's scores in place
-#pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8)
-          *reinterpret_cast<uint4*>(xrow + ((k8 ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * k8], pk[4 * k8 + 1], pk[4 * k8 + 2], pk[4 * k8 + 3]);
-        // cache slots past the sequence (or a page never loaded) feed the value
-        // product: zero their latent columns so that 0 * garbage cannot make NaN
-        if (nvalid < 64) {
-          unsigned char* pgb = pg_s + (jj % kStages) * kPageBytes;
-          const int nz = (64 - nvalid) * 4 * 8;          // 16-byte chunks to clear
-          for (int t = ltid; t < nz; t += 128) {
-            const int row = nvalid + t / 32, blk = (t / 8) & 3, ch = t & 7;
-            *reinterpret_cast<uint4*>(pgb + blk * 8192 + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
-          }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();  // orders an O rescale (tcgen05.st) before the value MMA
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->p_full[slot]);
+    while (ok && cb.next()) {
+      const int jj = cb.jj;
+      const int slot = jj & 1;
+      const int st = jj % kStages;
+      if (cb.first()) {
+        m_used = -INFINITY;
+        l = 0.f;
+        vis_last = a.seq_lens[cb.pc.b] - a.nq + qi;    // last key index this row may see
       }
-      if (!ok) break;
-
-      // epilogue: O / l and lse of this piece
-      const int jl = j + n - 1;
-      if (!wwait(&bar->o_done[jl & 1], (jl >> 1) & 1)) { ok = false; break; }
+      if (!wwait(&bar->s_full[slot], (jj >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const int grow_row = row0 + r;
-      float* dst = a.part_o + ((size_t)pc.id * prm.rows_total + grow_row) * a.d_c + c * 256;
-#pragma unroll 1
-      for (int cc = 0; cc < 256; cc += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_off + cc, o);
-        tmem_wait_ld();
-        if (row_valid) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + cc + i) =
-                make_float4(o[i] * inv_l, o[i + 1] * inv_l, o[i + 2] * inv_l, o[i + 3] * inv_l);
-        }
-      }
-      if (row_valid && c == 0)
-        a.part_lse[(size_t)pc.id * prm.rows_total + grow_row] =
-            l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      float s[64];
+      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off, s);
+      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32, s + 32);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->o_free);
-      j += n;
+      if (lane == 0) mbar_arrive(&bar->s_empty[slot]);
+      // the producer published the page's valid key count before its copy started
+      mbar_try_wait(&bar->pg_full[st], (jj / kStages) & 1);  // complete already: acquire only
+      const int nvalid = stage_nvalid[st];
+      const int lim_key = row_valid ? min(nvalid - 1, vis_last - cb.pg * 64) : -1;  // keys 0..lim_key visible
+      if (!wwait(&bar->x_full[slot], (jj >> 1) & 1)) { ok = false; break; }
+      const unsigned char* xrow = x_s + slot * kXBytes + r * 128;
+      float mx = -INFINITY;                            // scores carry a factor 2^-112 here
+#pragma unroll
+      for (int k8 = 0; k8 < 8; ++k8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xrow + ((k8 ^ (r & 7)) << 4));
+        const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i0 = 8 * k8 + 2 * e;
+          s[i0] = fmaf(s[i0], own_scale, h_lo_scaled(pv[e]));
+          s[i0 + 1] = fmaf(s[i0 + 1], own_scale, h_hi_scaled(pv[e]));
+        }
+      }
+      if (lim_key < 63) {                              // masked keys: past the length or causal
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s[i] = (i <= lim_key) ? s[i] : -INFINITY;
+      }
+      {
+        float t[16];                                   // tree reduction: short dependency chain
+#pragma unroll
+        for (int i = 0; i < 16; ++i) t[i] = fmaxf(fmaxf(s[i], s[i + 16]), fmaxf(s[i + 32], s[i + 48]));
+#pragma unroll
+        for (int n = 8; n > 0; n >>= 1)
+#pragma unroll
+          for (int i = 0; i < n; ++i) t[i] = fmaxf(t[i], t[i + n]);
+        mx = t[0] * kTwo112;
+      }
+
+      // lazy running max: rescale O and l only when the max grows by more than 2^8
+      const float m_new = fmaxf(m_used, mx);
+      const bool grow = m_new > m_used + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, grow && !cb.first() && m_used != -INFINITY)) {
+        const float alpha = (grow && m_used != -INFINITY) ? ex2(m_used - m_new) : 1.f;
+        const int jp = jj - 1;  // O must hold every earlier page of this piece
+        if (!wwait(&bar->o_done[jp & 1], (jp >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 256; cc += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_off + cc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tmem + lane_off + cc, o);
+        }
+        tmem_wait_st();
+        l *= alpha;
+      }
+      if (grow) m_used = m_new;
+      const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
+      uint32_t pk[32];
+      float ps[8];                                     // 8 partial sums: short dependency chains
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ps[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2(fmaf(s[2 * i], kTwo112, -m_ref));   // ex2(-inf) = 0
+        const float p1 = ex2(fmaf(s[2 * i + 1], kTwo112, -m_ref));
+        ps[i & 7] += p0 + p1;
+        pk[i] = pack_bf162(p0, p1);
+      }
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      // P(k) -> TMEM buffer (k & 1).  The value MMA of page k-2 read that buffer
+      // before the score MMA of page k ran (it is issued after it, in order), so
+      // the S(k) wait above already covers this reuse.
+      tmem_st32_bits(tmem + kTmemP + 32 * slot + lane_off, pk);
+      tmem_wait_st();
+      // cache slots past the sequence (or a page never loaded) feed the value
+      // product: zero their latent columns so that 0 * garbage cannot make NaN
+      if (nvalid < 64) {
+        unsigned char* pgb = pg_s + st * kPageBytes;
+        const int nz = (64 - nvalid) * 4 * 8;           // 16-byte chunks to clear
+        for (int t = ltid; t < nz; t += 128) {
+          const int row = nvalid + t / 32, blk = (t / 8) & 3, ch = t & 7;
+          *reinterpret_cast<uint4*>(pgb + blk * 8192 + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->p_full[slot]);
+
+      if (cb.last()) {
+        // epilogue: O / l and lse of this piece
+        if (!wwait(&bar->o_done[slot], (jj >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        const int grow_row = row0 + r;
+        float* dst = a.part_o + ((size_t)cb.pc.id * prm.rows_total + grow_row) * a.d_c + c * 256;
+#pragma unroll 1
+        for (int cc = 0; cc < 256; cc += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_off + cc, o);
+          tmem_wait_ld();
+          if (row_valid) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + cc + i) =
+                  make_float4(o[i] * inv_l, o[i + 1] * inv_l, o[i + 2] * inv_l, o[i + 3] * inv_l);
+          }
+        }
+        if (row_valid && c == 0)
+          a.part_lse[(size_t)cb.pc.id * prm.rows_total + grow_row] =
+              l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->o_free);
+      }
     }
   }
 
