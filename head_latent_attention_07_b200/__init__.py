@@ -42,6 +42,7 @@ SIGNATURES = {
     "mla_status_read": (ctypes.c_int, [_P, _P]),
     "mla_status_clear": (ctypes.c_int, [_P, _P]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mla_last_cuda_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_char_p)]),
     "mla_version": (ctypes.c_char_p, []),
 }
 
@@ -61,7 +62,12 @@ class MlaDims(ctypes.Structure):
 class MlaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} ({status})")
+        msg = f"{where}: {status_string(status)} ({status})"
+        if status == MLA_ERR_CUDA:
+            name = ctypes.c_char_p()
+            code = load_library().mla_last_cuda_error(ctypes.byref(name))
+            msg += f" [{name.value.decode() if name.value else '?'} ({code})]"
+        super().__init__(msg)
 
 
 _lib = None

@@ -38,11 +38,13 @@ float eff_scale(const mla_dims* d) {
 }
 float eff_theta(const mla_dims* d) { return d->rope_theta > 0.f ? d->rope_theta : kDefaultTheta; }
 
+int cuda_status(cudaError_t e);
+
 int device_sms(int* sms) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
-  return MLA_OK;
+  int st = cuda_status(cudaGetDevice(&dev));
+  if (st != MLA_OK) return st;
+  return cuda_status(cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev));
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -62,7 +64,13 @@ WsLayout ws_layout(const mla_dims* d, int batch, int nq, int sms) {
   return w;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;  // per calling host thread
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MLA_OK;
+  g_last_cuda_error = e;
+  return MLA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -156,9 +164,16 @@ int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16*
 int mla_status_read(const int32_t* dev_status, void* stream) {
   if (dev_status == nullptr) return MLA_ERR_INVALID_ARG;
   int32_t v = 0;
-  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
-  if (cudaMemcpy(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  int st = cuda_status(cudaStreamSynchronize((cudaStream_t)stream));
+  if (st != MLA_OK) return st;
+  if ((st = cuda_status(cudaMemcpy(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost))) != MLA_OK) return st;
   return v;
+}
+
+int mla_last_cuda_error(const char** name) {
+  const cudaError_t e = g_last_cuda_error;
+  if (name != nullptr) *name = cudaGetErrorName(e);
+  return (int)e;
 }
 
 int mla_status_clear(int32_t* dev_status, void* stream) {

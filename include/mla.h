@@ -204,6 +204,11 @@ int mla_status_read(const int32_t* dev_status, void* stream);
 /* mla_status_clear - reset the device word to MLA_OK (asynchronous on stream). */
 int mla_status_clear(int32_t* dev_status, void* stream);
 
+/* mla_last_cuda_error - the CUDA runtime error code behind the last MLA_ERR_CUDA
+ * returned to the calling host thread (0 if none); *name (if name is not NULL)
+ * receives its static name, e.g. "cudaErrorLaunchOutOfResources". */
+int mla_last_cuda_error(const char** name);
+
 /* mla_status_string - static description of an mla_status value. */
 const char* mla_status_string(int status);
 
