@@ -65,6 +65,37 @@ def algorithmic_counts(w: W.Workload, lens: np.ndarray) -> dict:
     return {"bytes": nbytes, "flops": flops, "cache_bytes": cache}
 
 
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_split_tc_v3.md")
+KERNEL_SOURCES = ["decode_tc.cu", "decode_combine.cu", "plan.cuh", "sm100.cuh", "common.cuh", "mma_frag.cuh",
+                  "decode.h"]
+
+
+def kernel_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(KERNEL_SOURCES):
+        h.update(f.encode())
+        with open(os.path.join(ROOT, "head_latent_attention_07_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload_name: str):
+    """DRAM bytes (read + write) of one mla_decode_attn call from the committed
+    ncu summary, or None when the summary is for another workload or the
+    kernel sources changed since it was taken."""
+    if workload_name != "v3" or not os.path.exists(PROFILE_SUMMARY):
+        return None, "no ncu capture for this workload"
+    fields = {}
+    for line in open(PROFILE_SUMMARY):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("sources_sha256") != kernel_sources_sha256():
+        return None, "kernel sources changed since the ncu capture"
+    return int(fields["traffic_bytes_per_call"]), "ncu dram__bytes_read.sum + dram__bytes_write.sum, split + combine"
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -273,8 +304,8 @@ class _Widen:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="v3", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
@@ -340,7 +371,7 @@ def main():
     roof = ({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s"} if bound == "hbm" else
             {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"})
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"], roof["traffic_source"] = profiled_traffic(w.name)
     roof["kernel"] = "mla_decode_attn (split + combine launches)"
     roof["peak_source"] = f"{src} (MEASURED_PEAKS.json burst figures)" if src == "measured" else "fallback"
     roof["hbm_frac"] = gbs / peaks["hbm_gbs"]
