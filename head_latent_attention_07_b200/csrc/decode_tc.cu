@@ -7,24 +7,30 @@
 // columns [256c, 256c + 256) and RoPE columns [512 + 32c, 512 + 32c + 32) of
 // every cache row and of the query tile, so each page is read from HBM once per
 // pair, half by each CTA.  Per page (64 tokens):
-//   GEMM1   S_c[128 x 64]  = Q_c[128 x 288] . K_c[64 x 288]^T        (tcgen05, TMEM)
-//   swap    each CTA scales S_c to log2 units, rounds it to fp16 and stores it
-//           into its peer's shared memory (st.async); each CTA then forms the
-//           full 576-wide score (content + RoPE) S = S_own + fp16(S_peer)
-//   softmax one thread per query row: running max / sum over the page, P in bf16
-//   GEMM2   O_c[128 x 256] += P[128 x 64] . C_c[64 x 256]               (tcgen05, TMEM)
-// The running max is only moved (and O rescaled in TMEM) when it grows by more
-// than 2^8; otherwise P is taken relative to the stale max (P <= 256).
-// TMEM: O_c uses columns [0, 256), the two S buffers [256, 320) and [320, 384).
+//   GEMM1   S_c[128 x 64] = Q_c[128 x 288] . K_c[64 x 288]^T: partial scores over
+//           this CTA's columns (latent part of Q_c in TMEM, RoPE part and the page
+//           in shared memory)
+//   swap    CTA c owns the softmax of keys [32c, 32c + 32) of every row: it sends
+//           the peer the partial scores of the peer's keys (fp16, log2 units) and
+//           adds the peer's partials of its own keys to its fp32 ones
+//   softmax the two CTAs agree on each row's running max (one float per row each
+//           way); each computes P (bf16) for its 32 keys and writes it into both
+//           CTAs' P tiles
+//   GEMM2   O_c[128 x 256] += P[128 x 64] . C_c[64 x 256]  (P and page in shared
+//           memory, O in TMEM)
+// The running max is only moved (and O rescaled in TMEM, by both CTAs alike) when
+// it grows by more than 2^8; otherwise P is taken relative to the stale max.
+// Each CTA keeps the row sums of its own keys; the two halves are added at the
+// end of every piece, and each CTA normalises its own 256 columns of O.
+// TMEM: O columns [0, 256), S buffers [256, 320) and [320, 384), Q latent
+// (bf16 pairs) [384, 512).
 //
-// Warp roles (448 threads): warp 0 lane 0 issues TMA loads (query tile once per
-// piece, pages into a 3-stage ring, L2 prefetch further ahead), warp 1 owns TMEM
-// and lane 0 issues the MMAs (score GEMM up to two pages ahead of the value
-// GEMM), warps 2..5 (one per TMEM lane quarter) send this CTA's partial scores to
-// the peer, and warps 6..9 (one per lane quarter, one query row per thread) run
-// the softmax and epilogue.  Each CTA adds its own fp32 partial scores to the
-// peer's fp16 ones; the two CTAs' scores differ only by that rounding, and each
-// normalises its own half of O with its own running sum.
+// Warp roles (320 threads): warp 0 lane 0 issues TMA loads (RoPE part of the
+// query tile once per piece, pages into a 4-stage ring, L2 prefetch further
+// ahead), warp 1 owns TMEM and lane 0 issues the MMAs, warps 2..5 (one per TMEM
+// lane quarter, one query row per thread) load the query tile's latent part into
+// TMEM and send the peer its partial scores, and warps 6..9 (same layout) run the
+// softmax and the epilogue.
 // Every mbarrier wait is bounded: on time-out the kernel records MLA_ERR_TIMEOUT,
 // stops its loops, drains its own copies and MMAs and frees TMEM.
 #include <cuda.h>
@@ -43,27 +49,30 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;  // producer, MMA, 4 exchange warps, 4 softmax warps
-constexpr int kStages = 3;
+constexpr int kThreads = 320;  // producer, MMA, 4 sender warps, 4 softmax warps
+constexpr int kStages = 4;
 constexpr int kPrefetch = 4;  // pages beyond the shared-memory ring prefetched into L2
-constexpr int kQBytes = 4 * 16384 + 8192;     // 4 latent blocks [128 x 64] + RoPE block [128 x 32]
-constexpr int kPageBytes = 4 * 8192 + 4096;   // 4 latent blocks [64 x 64]  + RoPE block [64 x 32]
-constexpr int kXBytes = 128 * 128;            // [128 rows x 64] fp16 scores, then bf16 P
-constexpr int kOffQ = 0;
-constexpr int kOffPg = kOffQ + kQBytes;
+constexpr int kQrBytes = 128 * 64;            // RoPE block of the query tile [128 x 32] (64-byte swizzle)
+constexpr int kPageBytes = 4 * 8192 + 4096;   // 4 latent blocks [64 x 64] + RoPE block [64 x 32]
+constexpr int kXBytes = 128 * 64;             // received partial scores: [128 rows x 32 keys] fp16
+constexpr int kPBytes = 128 * 128;            // P tile [128 rows x 64 keys] bf16, 128-byte swizzle
+constexpr int kOffQr = 0;
+constexpr int kOffPg = kOffQr + kQrBytes;
 constexpr int kOffX = kOffPg + kStages * kPageBytes;
-constexpr int kOffPlan = kOffX + 2 * kXBytes;
+constexpr int kOffP = kOffX + 2 * kXBytes;
+constexpr int kOffM = kOffP + 2 * kPBytes;    // received row maxima [2][128], row sums [128] (fp32)
+constexpr int kOffPlan = kOffM + 3 * 128 * 4;
 constexpr int kOffBar = kOffPlan + ((int(sizeof(PlanSmem)) + 127) & ~127);
-constexpr int kNumBars = 24;
+constexpr int kNumBars = 32;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;       // TMEM base, abort flag, page metadata
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;       // + 1 KB alignment slack
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: rescale when the max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 256;              // S buffers: columns [256, 320) and [320, 384)
-constexpr uint32_t kTmemP = 384;              // P buffers (bf16 pairs): [384, 416) and [416, 448)
+constexpr uint32_t kTmemQ = 384;              // Q latent, 256 bf16 per row: columns [384, 512)
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffPg % 1024 == 0 && kPageBytes % 1024 == 0 && kOffX % 1024 == 0, "swizzle alignment");
+static_assert(kOffPg % 1024 == 0 && kPageBytes % 1024 == 0 && kOffP % 1024 == 0, "swizzle alignment");
 
 struct TcParams {
   DecodeArgs d;
@@ -76,9 +85,11 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t pg_full[kStages], pg_empty[kStages];
   uint64_t s_full[2], s_empty[2];
-  uint64_t x_full[2], x_free[2];
-  uint64_t p_full[2], o_done[2];
-  uint64_t o_free, drain;
+  uint64_t x_full[2], x_free[2];   // partial scores from the peer / the peer's slot is free
+  uint64_t m_full[2];              // the peer's row maxima of a page
+  uint64_t p_full[2], p_free[2];   // P tile complete (own + peer half) / the peer's P tile is free
+  uint64_t o_done[2];
+  uint64_t l_full, o_free, drain;
 };
 static_assert(sizeof(Bars) <= kNumBars * 8, "barrier area");
 
@@ -143,9 +154,6 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ float2 unpack_half2(uint32_t v) {
-  return __half22float2(*reinterpret_cast<__half2*>(&v));
-}
 __device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -163,15 +171,17 @@ __device__ __forceinline__ float h_hi_scaled(uint32_t v) {
 constexpr float kTwo112 = 5.192296858534828e33f;  // 2^112
 
 __global__ void __launch_bounds__(kThreads, 1)
-decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_constant__ CUtensorMap tq64,
-                       const __grid_constant__ CUtensorMap tp128, const __grid_constant__ CUtensorMap tp64,
-                       const TcParams prm) {
+decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_constant__ CUtensorMap tp128,
+                       const __grid_constant__ CUtensorMap tp64, const TcParams prm) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* q_s = sm + kOffQ;
+  unsigned char* qr_s = sm + kOffQr;
   unsigned char* pg_s = sm + kOffPg;
   unsigned char* x_s = sm + kOffX;
+  unsigned char* p_s = sm + kOffP;
+  float* m_recv = reinterpret_cast<float*>(sm + kOffM);         // [2][128]
+  float* l_recv = m_recv + 256;                                 // [128]
   PlanSmem* plan = reinterpret_cast<PlanSmem*>(sm + kOffPlan);
   Bars* bar = reinterpret_cast<Bars*>(sm + kOffBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + kOffMisc);
@@ -189,24 +199,27 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
   int32_t* status = a.dev_status;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_full, 5);        // 4 sender warps (latent part) + producer (RoPE part, bytes)
     mbar_init(&bar->q_empty, 1);
     for (int s = 0; s < kStages; ++s) { mbar_init(&bar->pg_full[s], 1); mbar_init(&bar->pg_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->s_empty[s], 8);   // 4 exchange warps + 4 softmax warps read S
-      mbar_init(&bar->x_full[s], 1);
-      mbar_init(&bar->x_free[s], 1);   // the peer's value MMA of the page ran: its slot was read
-      mbar_init(&bar->p_full[s], 4);
+      mbar_init(&bar->s_empty[s], 8);  // 4 sender warps + 4 softmax warps read S
+      mbar_init(&bar->x_full[s], 1);   // local softmax leader's expect-bytes arrival; the peer's stores carry the bytes
+      mbar_init(&bar->x_free[s], 4);   // the peer's 4 softmax warps have read their slot
+      mbar_init(&bar->m_full[s], 1);
+      mbar_init(&bar->p_full[s], 4);   // 4 local softmax warps (one also expects the peer's bytes)
+      mbar_init(&bar->p_free[s], 1);   // the peer's value MMA of the page has read its P tile
       mbar_init(&bar->o_done[s], 1);
     }
+    mbar_init(&bar->l_full, 1);
     mbar_init(&bar->o_free, 4);
     mbar_init(&bar->drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch(&tq128); tma_prefetch(&tq64); tma_prefetch(&tp128); tma_prefetch(&tp64);
+    tma_prefetch(&tq64); tma_prefetch(&tp128); tma_prefetch(&tp64);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, kTmemCols);
@@ -235,7 +248,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
         more_pf = pf.next();
       };
       for (int i = 0; i < kStages + kPrefetch; ++i) prefetch_next();
-      int issued[kStages] = {0, 0, 0}, issued_q = 0;
+      int issued[kStages] = {0, 0, 0, 0}, issued_q = 0;
       bool more = cu.next();
       int id_next = more ? a.page_table[(size_t)cu.pc.b * a.max_pages + cu.pg] : 0;
       int len_next = more ? a.seq_lens[cu.pc.b] : 0;
@@ -246,9 +259,8 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
         if (cu.first()) {
           if (cu.p > 0 && !mbar_wait(&bar->q_empty, (cu.p - 1) & 1, abort_flag, status, lim)) break;
           const int qrow = cu.pc.b * prm.rows_total + row0;
-          mbar_arrive_expect_tx(&bar->q_full, kQBytes);
-          for (int i = 0; i < 4; ++i) tma_load_2d(q_s + i * 16384, &tq128, c * 256 + 64 * i, qrow, &bar->q_full);
-          tma_load_2d(q_s + 65536, &tq64, 512 + 32 * c, qrow, &bar->q_full);
+          mbar_arrive_expect_tx(&bar->q_full, kQrBytes);
+          tma_load_2d(qr_s, &tq64, 512 + 32 * c, qrow, &bar->q_full);
           ++issued_q;
         }
         const int st = jj % kStages;
@@ -281,43 +293,46 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Two in-order queues: GEMM1 (scores, up to two pages ahead) and GEMM2
-    // (values); each is issued as soon as its own inputs are ready.
+    // Two in-order queues, each issued as soon as its inputs are ready: GEMM1
+    // (scores, up to two pages ahead: S is double-buffered) and GEMM2 (values,
+    // checked first).
     if (lane == 0) {
       const uint32_t id1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id2 = idesc_bf16_f32(128, 256, 0, 1);
-      const uint32_t qa = smem_u32(q_s);
+      const uint32_t qra = smem_u32(qr_s);
       PageCursor g1(plan, a.batch, w), g2(plan, a.batch, w);
       bool has1 = g1.next(), has2 = g2.next();
       bool q_ok = false;  // query tile of g1's piece is resident
+      int last2 = -1;     // last page whose value MMAs were issued
       long long t_last = clock64();
       while (has1 || has2) {
         bool progressed = false;
-        if (has2 && g2.jj < (has1 ? g1.jj : 0x7fffffff)) {
+        if (has2 && (!has1 || g2.jj < g1.jj)) {
           const int jj = g2.jj;
           const bool first = g2.first();
           const bool ready = (!(first && g2.p > 0) || mbar_test(&bar->o_free, (g2.p - 1) & 1)) &&
                              mbar_test(&bar->p_full[jj & 1], (jj >> 1) & 1);
           if (ready) {
+            fence_proxy_async_smem();  // P written by threads of both CTAs, read by the tensor core
             tc_fence_after();
-            const uint32_t pa = tmem + kTmemP + 32 * (jj & 1);
+            const uint32_t pa = smem_u32(p_s + (jj & 1) * kPBytes);
             const uint32_t pb = smem_u32(pg_s + (jj % kStages) * kPageBytes);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t da = smem_desc(pa + ks * 32, 16, 1024, kSwizzle128);
               const uint64_t db = smem_desc(pb + ks * 2048, 8192, 1024, kSwizzle128);
-              mma_bf16_ts(tmem, pa + 8 * ks, db, id2, (first && ks == 0) ? 0u : 1u);
+              mma_bf16(tmem, da, db, id2, (first && ks == 0) ? 0u : 1u);
             }
             mma_commit(&bar->pg_empty[jj % kStages]);
             mma_commit(&bar->o_done[jj & 1]);
-            // this CTA's receive slot (jj & 1) has been read: the peer may send page jj + 2
-            mma_commit_mc(&bar->x_free[jj & 1], uint16_t(1u << peer));
+            // this CTA's P tile (jj & 1) has been read: the peer may write page jj + 2's half
+            mma_commit_mc(&bar->p_free[jj & 1], uint16_t(1u << peer));
+            last2 = jj;
             has2 = g2.next();
             progressed = true;
           }
         }
-        // GEMM1(j) waits for GEMM2(j - 2) to be issued: the tensor pipe runs in
-        // order, and the value product gates more of the pipeline than the scores
-        if (has1 && (!has2 || g1.jj < g2.jj + 2)) {
+        if (has1) {
           const int jj = g1.jj;
           const int st = jj % kStages;
           if (g1.first() && !q_ok) q_ok = mbar_test(&bar->q_full, g1.p & 1);
@@ -329,16 +344,15 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
             const uint32_t pb = smem_u32(pg_s + st * kPageBytes);
             const uint32_t ts = tmem + kTmemS + 64 * (jj & 1);
 #pragma unroll
-            for (int ks = 0; ks < 18; ++ks) {
-              uint64_t da, db;
-              if (ks < 16) {
-                da = smem_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwizzle128);
-                db = smem_desc(pb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128);
-              } else {
-                da = smem_desc(qa + 65536 + (ks - 16) * 32, 16, 512, kSwizzle64);
-                db = smem_desc(pb + 32768 + (ks - 16) * 32, 16, 512, kSwizzle64);
-              }
-              mma_bf16(ts, da, db, id1, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 16; ++ks) {          // latent part: A from TMEM
+              const uint64_t db = smem_desc(pb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128);
+              mma_bf16_ts(ts, tmem + kTmemQ + 8 * ks, db, id1, ks > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {           // RoPE part: A from shared memory
+              const uint64_t da = smem_desc(qra + ks * 32, 16, 512, kSwizzle64);
+              const uint64_t db = smem_desc(pb + 32768 + ks * 32, 16, 512, kSwizzle64);
+              mma_bf16(ts, da, db, id1, 1u);
             }
             mma_commit(&bar->s_full[jj & 1]);
             if (g1.last()) {
@@ -362,52 +376,85 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
       // drain: every MMA issued above has completed before TMEM / smem go away
       mma_commit(&bar->drain);
       mbar_wait_drain(&bar->drain, 0, lim);
+      // the peer's value MMAs of the last two pages release this CTA's P tiles by
+      // a multicast arrive that nothing else waits for: let it land
+      const long long lim_drain = *abort_flag ? (1ll << 20) : lim;
+      for (int jj = max(0, last2 - 1); jj <= last2; ++jj)
+        mbar_wait_drain(&bar->p_free[jj & 1], (jj >> 1) & 1, lim_drain);
     }
   } else if (warp < 6) {
-    // ------------------------------------------------------------ exchange warps
-    // A(k): this CTA's partial scores S(k) out of TMEM, scaled to log2 units,
-    // rounded to fp16 and stored into the peer's receive slot (k & 1).  Runs up
-    // to two pages ahead of the softmax warps.
+    // ------------------------------------------------------------ sender warps
+    // Per piece: the latent part of this CTA's query columns into TMEM.  Per
+    // page: the partial scores of the peer's keys out of TMEM, scaled to log2
+    // units, rounded to fp16 and stored into the peer's receive slot (k & 1).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t x_peer = mapa(smem_u32(x_s), peer);
     const uint32_t xfull_peer = mapa(smem_u32(&bar->x_full[0]), peer);
+    const uint32_t sw = uint32_t((r >> 1) & 3);        // chunk swizzle of row r in a receive slot
     auto wwait = [&](uint64_t* b, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, status, lim));
     };
     PageCursor ca(plan, a.batch, w);
+    int last_jj = -1;
     while (ca.next()) {
       const int jj = ca.jj;
       const int slot = jj & 1;
+      if (ca.first()) {
+        // the previous piece's score MMAs are done with TMEM's query columns
+        if (ca.p > 0 && !wwait(&bar->q_empty, (ca.p - 1) & 1)) break;
+        const uint16_t* qsrc = a.q_lat + ((size_t)ca.pc.b * prm.rows_total + row0 + r) * 576 + 256 * c;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {                // 64 bf16 = 32 TMEM columns per chunk
+          uint32_t v[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 u = r < rows_valid ? ldg_stream(qsrc + 64 * cc + 8 * i) : make_uint4(0, 0, 0, 0);
+            v[4 * i] = u.x; v[4 * i + 1] = u.y; v[4 * i + 2] = u.z; v[4 * i + 3] = u.w;
+          }
+          tmem_st32_bits(tmem + lane_off + kTmemQ + 32 * cc, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->q_full);
+      }
       if (!wwait(&bar->s_full[slot], (jj >> 1) & 1)) break;
       tc_fence_after();
-      float sv[64];
-      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off, sv);
-      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32, sv + 32);
+      float sv[32];
+      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32 * peer, sv);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->s_empty[slot]);
-      uint32_t h[32];
+      uint32_t h[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) h[i] = pack_half2(sv[2 * i] * prm.scale_log2, sv[2 * i + 1] * prm.scale_log2);
+      for (int i = 0; i < 16; ++i) h[i] = pack_half2(sv[2 * i] * prm.scale_log2, sv[2 * i + 1] * prm.scale_log2);
       // the peer's receive slot is free once its softmax warps have read page jj - 2
       if (jj >= 2 && !wwait(&bar->x_free[slot], ((jj >> 1) - 1) & 1)) break;
-      const uint32_t dst = x_peer + slot * kXBytes + r * 128;
+      const uint32_t dst = x_peer + slot * kXBytes + r * 64;
       const uint32_t rbar = xfull_peer + slot * 8;
 #pragma unroll
-      for (int k8 = 0; k8 < 8; ++k8)
-        st_async_v4(dst + ((k8 ^ (r & 7)) << 4), make_uint4(h[4 * k8], h[4 * k8 + 1], h[4 * k8 + 2], h[4 * k8 + 3]),
+      for (int k4 = 0; k4 < 4; ++k4)
+        st_async_v4(dst + ((k4 ^ sw) << 4), make_uint4(h[4 * k4], h[4 * k4 + 1], h[4 * k4 + 2], h[4 * k4 + 3]),
                     rbar);
-      if (warp == 2 && lane == 0) mbar_arrive_expect_tx(&bar->x_full[slot], kXBytes);
+      last_jj = jj;
+    }
+    // the peer's softmax warps release the last two slots after this loop ends:
+    // their arrivals must land before this CTA's shared memory is released
+    if (warp == 2 && lane == 0) {
+      const long long lim_drain = *abort_flag ? (1ll << 20) : lim;
+      for (int jj = max(0, last_jj - 1); jj <= last_jj; ++jj)
+        mbar_wait_drain(&bar->x_free[jj & 1], (jj >> 1) & 1, lim_drain);
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    // B(k), one query row per thread, all 64 keys of the page:
+    // B(k), one query row per thread, this CTA's 32 keys of the page:
     //   S = own + peer: this CTA's fp32 partial (scaled) plus the peer's fp16 one,
-    //   masked online softmax, P(k) (bf16) into TMEM, O rescale when the max grew,
-    //   epilogue (O / l, lse) at the end of each piece.
+    //   masked; the row max is agreed with the peer (both take the max of the two
+    //   halves), P(k) (bf16) goes into both CTAs' P tiles, O is rescaled when the
+    //   max grew, epilogue (O / l, lse) at the end of each piece.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                 // query row within the tile = TMEM lane
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
@@ -415,6 +462,15 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
     const int qi = (row0 + r) / a.n_heads;             // query token of this row
     const int ltid = threadIdx.x - 192;                // 0..127
     const float own_scale = prm.scale_log2 * (1.0f / kTwo112);  // own partial in the peer's 2^-112 units
+    const uint32_t sw = uint32_t((r >> 1) & 3);
+    const uint32_t xfree_peer = mapa(smem_u32(&bar->x_free[0]), peer);
+    const uint32_t mrecv_peer = mapa(smem_u32(m_recv), peer);
+    const uint32_t mfull_peer = mapa(smem_u32(&bar->m_full[0]), peer);
+    const uint32_t lrecv_peer = mapa(smem_u32(l_recv), peer);
+    const uint32_t lfull_peer = mapa(smem_u32(&bar->l_full), peer);
+    const uint32_t p_peer = mapa(smem_u32(p_s), peer);
+    const uint32_t pfull_peer = mapa(smem_u32(&bar->p_full[0]), peer);
+    const bool leader = warp == 6 && lane == 0;        // posts the expected byte counts
     auto wwait = [&](uint64_t* b, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, status, lim));
     };
@@ -434,9 +490,8 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
       }
       if (!wwait(&bar->s_full[slot], (jj >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      float s[64];
-      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off, s);
-      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32, s + 32);
+      float s[32];
+      tmem_ld32(tmem + kTmemS + 64 * slot + lane_off + 32 * c, s);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -444,35 +499,48 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
       // the producer published the page's valid key count before its copy started
       mbar_try_wait(&bar->pg_full[st], (jj / kStages) & 1);  // complete already: acquire only
       const int nvalid = stage_nvalid[st];
-      const int lim_key = row_valid ? min(nvalid - 1, vis_last - cb.pg * 64) : -1;  // keys 0..lim_key visible
+      // keys 32c + [0, lim_h] are visible to this row
+      const int lim_h = (row_valid ? min(nvalid - 1, vis_last - cb.pg * 64) : -1) - 32 * (int)c;
+      // the peer's partial scores of this CTA's keys; the expected byte count is
+      // posted by the consumer, once the slot's previous phase has completed
+      if (leader) mbar_arrive_expect_tx(&bar->x_full[slot], kXBytes);
       if (!wwait(&bar->x_full[slot], (jj >> 1) & 1)) { ok = false; break; }
-      const unsigned char* xrow = x_s + slot * kXBytes + r * 128;
-      float mx = -INFINITY;                            // scores carry a factor 2^-112 here
+      const unsigned char* xrow = x_s + slot * kXBytes + r * 64;
 #pragma unroll
-      for (int k8 = 0; k8 < 8; ++k8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(xrow + ((k8 ^ (r & 7)) << 4));
+      for (int k4 = 0; k4 < 4; ++k4) {                 // scores carry a factor 2^-112 here
+        const uint4 v = *reinterpret_cast<const uint4*>(xrow + ((k4 ^ sw) << 4));
         const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i0 = 8 * k8 + 2 * e;
+          const int i0 = 8 * k4 + 2 * e;
           s[i0] = fmaf(s[i0], own_scale, h_lo_scaled(pv[e]));
           s[i0 + 1] = fmaf(s[i0 + 1], own_scale, h_hi_scaled(pv[e]));
         }
       }
-      if (lim_key < 63) {                              // masked keys: past the length or causal
+      // the peer may refill this slot: the loads above have returned (their values
+      // are consumed), so the arrive needs no release ordering
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + slot * 8);
+      if (lim_h < 31) {                                // masked keys: past the length or causal
 #pragma unroll
-        for (int i = 0; i < 64; ++i) s[i] = (i <= lim_key) ? s[i] : -INFINITY;
+        for (int i = 0; i < 32; ++i) s[i] = (i <= lim_h) ? s[i] : -INFINITY;
       }
+      float mx;
       {
-        float t[16];                                   // tree reduction: short dependency chain
+        float t[8];                                    // tree reduction: short dependency chain
 #pragma unroll
-        for (int i = 0; i < 16; ++i) t[i] = fmaxf(fmaxf(s[i], s[i + 16]), fmaxf(s[i + 32], s[i + 48]));
+        for (int i = 0; i < 8; ++i) t[i] = fmaxf(fmaxf(s[i], s[i + 8]), fmaxf(s[i + 16], s[i + 24]));
 #pragma unroll
-        for (int n = 8; n > 0; n >>= 1)
+        for (int n = 4; n > 0; n >>= 1)
 #pragma unroll
           for (int i = 0; i < n; ++i) t[i] = fmaxf(t[i], t[i + n]);
         mx = t[0] * kTwo112;
       }
+      // swap the row maxima of the two key halves with the peer
+      if (leader) mbar_arrive_expect_tx(&bar->m_full[slot], 128 * 4);
+      st_async_b32(mrecv_peer + (slot * 128 + r) * 4, __float_as_uint(mx), mfull_peer + slot * 8);
+      if (!wwait(&bar->m_full[slot], (jj >> 1) & 1)) { ok = false; break; }
+      mx = fmaxf(mx, m_recv[slot * 128 + r]);          // both CTAs now hold the same row max
 
       // lazy running max: rescale O and l only when the max grows by more than 2^8
       const float m_new = fmaxf(m_used, mx);
@@ -496,23 +564,35 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
       }
       if (grow) m_used = m_new;
       const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t pk[32];
-      float ps[8];                                     // 8 partial sums: short dependency chains
+      uint32_t pk[16];
+      float ps[4];                                     // 4 partial sums: short dependency chains
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ps[i] = 0.f;
+      for (int i = 0; i < 4; ++i) ps[i] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const float p0 = ex2(fmaf(s[2 * i], kTwo112, -m_ref));   // ex2(-inf) = 0
         const float p1 = ex2(fmaf(s[2 * i + 1], kTwo112, -m_ref));
-        ps[i & 7] += p0 + p1;
+        ps[i & 3] += p0 + p1;
         pk[i] = pack_bf162(p0, p1);
       }
-      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      // P(k) -> TMEM buffer (k & 1).  The value MMA of page k-2 read that buffer
-      // before the score MMA of page k ran (it is issued after it, in order), so
-      // the S(k) wait above already covers this reuse.
-      tmem_st32_bits(tmem + kTmemP + 32 * slot + lane_off, pk);
-      tmem_wait_st();
+      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      // P(k) -> P tile (k & 1) of both CTAs, keys [32c, 32c + 32) of row r, once
+      // the value MMAs of page k - 2 (own and peer) have read those tiles
+      if (jj >= 2) {
+        if (!wwait(&bar->o_done[slot], ((jj >> 1) - 1) & 1)) { ok = false; break; }
+        if (!wwait(&bar->p_free[slot], ((jj >> 1) - 1) & 1)) { ok = false; break; }
+      }
+      {
+        const uint32_t prow = slot * kPBytes + r * 128;
+        unsigned char* own = p_s + prow;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const uint32_t off = ((4 * c + k4) ^ (r & 7)) << 4;   // 128-byte swizzle of the UMMA K-major tile
+          const uint4 v = make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
+          *reinterpret_cast<uint4*>(own + off) = v;
+          st_async_v4(p_peer + prow + off, v, pfull_peer + slot * 8);
+        }
+      }
       // cache slots past the sequence (or a page never loaded) feed the value
       // product: zero their latent columns so that 0 * garbage cannot make NaN
       if (nvalid < 64) {
@@ -522,17 +602,24 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
           const int row = nvalid + t / 32, blk = (t / 8) & 3, ch = t & 7;
           *reinterpret_cast<uint4*>(pgb + blk * 8192 + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
         }
-        fence_proxy_async_smem();
       }
+      fence_proxy_async_smem();                        // own P / zeroed rows -> tensor core
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->p_full[slot]);
+      if (lane == 0) {
+        if (warp == 6) mbar_arrive_expect_tx(&bar->p_full[slot], kPBytes / 2);  // the peer's half
+        else mbar_arrive(&bar->p_full[slot]);
+      }
 
       if (cb.last()) {
-        // epilogue: O / l and lse of this piece
+        // epilogue: O / l and lse of this piece, l summed over the two key halves
+        if (leader) mbar_arrive_expect_tx(&bar->l_full, 128 * 4);
+        st_async_b32(lrecv_peer + r * 4, __float_as_uint(l), lfull_peer);
+        if (!wwait(&bar->l_full, cb.p & 1)) { ok = false; break; }
+        const float lt = l + l_recv[r];
         if (!wwait(&bar->o_done[slot], (jj >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
         const int grow_row = row0 + r;
         float* dst = a.part_o + ((size_t)cb.pc.id * prm.rows_total + grow_row) * a.d_c + c * 256;
 #pragma unroll 1
@@ -549,7 +636,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
         }
         if (row_valid && c == 0)
           a.part_lse[(size_t)cb.pc.id * prm.rows_total + grow_row] =
-              l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+              lt > 0.f ? (m_used + log2f(lt)) * 0.6931471805599453f : -INFINITY;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->o_free);
@@ -562,6 +649,12 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq128, const __grid_c
   __syncthreads();
   __syncwarp();
   cluster_sync();  // the peer no longer stores into this CTA's shared memory
+  if (*abort_flag) {
+    // after a time-out the peer may have stores to this CTA still in flight
+    // (its waits for them gave up): give them time to land before exiting
+    const long long t0 = clock64();
+    while (clock64() - t0 < 200000) __nanosleep(1000);
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -613,11 +706,10 @@ int decode_tc_workers(int sms, int rows_total) {
 
 cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cudaStream_t stream) {
   const int rows_total = a.nq * a.n_heads;
-  CUtensorMap tq128, tq64, tp128, tp64;
+  CUtensorMap tq64, tp128, tp64;
   const uint64_t qrows = (uint64_t)a.batch * rows_total;
   const uint64_t prows = (uint64_t)a.num_pages * 64;
-  if (!encode_rows576(&tq128, a.q_lat, qrows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_rows576(&tq64, a.q_lat, qrows, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
+  if (!encode_rows576(&tq64, a.q_lat, qrows, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !encode_rows576(&tp128, a.pool, prows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_rows576(&tp64, a.pool, prows, 32, 64, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
@@ -641,7 +733,7 @@ cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cu
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_split_tc_kernel, tq128, tq64, tp128, tp64, prm);
+  e = cudaLaunchKernelEx(&cfg, decode_split_tc_kernel, tq64, tp128, tp64, prm);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
