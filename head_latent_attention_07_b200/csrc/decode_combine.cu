@@ -5,11 +5,15 @@
 //   o_lat = sum_s exp(lse_s - LSE) * O_s          (O_s already normalised per piece)
 //   out[t][h][v] = sum_c W_UV[h][v][c] * o_lat[c]  (values up-projected once, after
 //                                                   attending over latents)
-// One CTA = one head and up to 16 query tokens.  The merge runs on all 256
-// threads (coalesced reads of the partials); the up-projection is a
-// [v_head x d_c] x [d_c x 16] product on the tensor cores (mma.sync, fp32
-// accumulate) with o_lat split into two bf16 terms (hi + lo), which keeps about
-// 16 bits of its mantissa.  W_UV,h is streamed once per group of 16 tokens.
+// Work split: a cluster of KS = ceil(d_c / 128) CTAs per (head, group of 16
+// query tokens); CTA ks owns latent columns [128 ks, 128 ks + 128).  It merges
+// its columns of the partials (each partial byte is read once, by one CTA) and
+// multiplies them by its 128-column slice of W_UV,h on the tensor cores
+// (mma.sync, fp32 accumulate, o_lat split into two bf16 terms, hi + lo, which
+// keeps about 16 bits of its mantissa).  The KS partial products are summed
+// through distributed shared memory, each CTA finishing 1/KS of the rows of
+// out.  Many small CTAs keep enough loads in flight to stream the partials and
+// W_UV at memory speed.
 #include "common.cuh"
 #include "decode.h"
 #include "mma_frag.cuh"
@@ -20,152 +24,215 @@ namespace mla {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTok = 16;
+constexpr int kTok = 16;       // query tokens per CTA
+constexpr int kSlice = 128;    // latent columns per CTA
+constexpr int kVChunk = 128;   // out rows reduced per cluster round
+constexpr int kOStride = kSlice + 8;   // bf16 row stride of the merged slice (16-byte pad)
+constexpr int kPieceBatch = 6;         // pieces whose loads are in flight at once
 
-__device__ __forceinline__ uint4 ld_nc_v4(const uint16_t* p) { return ldg_stream(p); }
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t local_smem, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_smem), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
 
-__global__ void __launch_bounds__(kThreads)
-decode_combine_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 2)
+decode_combine_kernel(DecodeArgs a, int KS) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PlanSmem* ps = reinterpret_cast<PlanSmem*>(smem_raw);
-  const int kpad = ((a.d_c + 31) & ~31);                 // reduction length padded to 32
-  const int ostride = kpad + 8;                          // bf16 row stride (16-byte pad: no bank conflicts)
   uint16_t* o_hi = reinterpret_cast<uint16_t*>(smem_raw + ((sizeof(PlanSmem) + 15) & ~size_t(15)));
-  uint16_t* o_lo = o_hi + kTok * ostride;
+  uint16_t* o_lo = o_hi + kTok * kOStride;
+  float* red = reinterpret_cast<float*>(o_lo + kTok * kOStride);   // [kVChunk][kTok] partial products
 
   build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr);
   const int h = blockIdx.x;
-  const int t0 = blockIdx.y * kTok;
+  const int ks = (int)cta_rank();
+  const int t0 = (blockIdx.y / KS) * kTok;
   const int T = a.batch * a.nq;
   const int rows_total = a.nq * a.n_heads;
+  const int col0 = ks * kSlice;
+  const int ncol = min(kSlice, a.d_c - col0);   // multiple of 8
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // 1. merge: 16 threads per token, each owning 8 consecutive columns per 128
+  // this slice's weights for the first chunk of out rows, loaded before the
+  // merge so that their latency overlaps it (see step 2 for the fragment layout)
+  const int g = lane >> 2, q = lane & 3;
+  const uint16_t* wh = a.w_uv + (size_t)h * a.v_head * a.d_c + col0;
+  uint4 ra[4], rb[4];
+  auto load_w = [&](int v0) {
+    const int va = v0 + warp * 16 + g, vb = va + 8;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {                   // four 32-wide k slices in flight
+      const int kk = 32 * u + 8 * q;
+      const bool kin = kk < ncol;
+      ra[u] = (kin && va < a.v_head) ? ldg_stream(wh + (size_t)va * a.d_c + kk) : z;
+      rb[u] = (kin && vb < a.v_head) ? ldg_stream(wh + (size_t)vb * a.d_c + kk) : z;
+    }
+  };
+  load_w(0);
+
+  // 1. merge: 16 threads per token, each owning 8 consecutive columns of the
+  //    slice; one pass over the pieces in batches of 8 (their LSEs and partial
+  //    rows loaded together), with the running max moved as batches arrive
   {
-    const int j = tid >> 4, sub = tid & 15;
+    const int j = tid >> 4, gc = tid & 15;
     const int t = t0 + j;
-    float lse_all = -INFINITY;
-    int pb = 0, np = 0, row = 0;
+    const int c0 = 8 * gc;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     if (t < T) {
       const int b = t / a.nq, i = t % a.nq;
-      row = i * a.n_heads + h;
-      pb = ps->piece_begin[b];
-      np = ps->piece_begin[b + 1] - pb;
-      float mx = -INFINITY;
-      for (int s = 0; s < np; ++s) mx = fmaxf(mx, a.part_lse[(size_t)(pb + s) * rows_total + row]);
-      if (mx != -INFINITY) {
-        float tot = 0.f;
-        for (int s = 0; s < np; ++s) {
-          const float l = a.part_lse[(size_t)(pb + s) * rows_total + row];
-          tot += (l == -INFINITY) ? 0.f : expf(l - mx);
-        }
-        lse_all = mx + logf(tot);
-      }
-      if (sub == 0 && a.lse != nullptr) a.lse[(size_t)t * a.n_heads + h] = lse_all;
-    }
-    for (int c0 = sub * 8; c0 < kpad; c0 += 128) {
-      float acc[8];
+      const int row = i * a.n_heads + h;
+      const int pb = ps->piece_begin[b];
+      const int np = ps->piece_begin[b + 1] - pb;
+      const bool cols = c0 < ncol;
+      float m = -INFINITY, tot = 0.f;
+      for (int s0 = 0; s0 < np; s0 += kPieceBatch) {
+        float lv[kPieceBatch];
+        float4 v0[kPieceBatch], v1[kPieceBatch];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-      if (lse_all != -INFINITY && c0 < a.d_c) {
-        for (int s0 = 0; s0 < np; s0 += 4) {         // four pieces' loads in flight at once
-          float4 v0[4], v1[4];
-          float wgt[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int s = s0 + u;
-            wgt[u] = 0.f;
-            v0[u] = v1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (s < np) {
-              const float l = a.part_lse[(size_t)(pb + s) * rows_total + row];
-              const float* src = a.part_o + ((size_t)(pb + s) * rows_total + row) * a.d_c + c0;
-              v0[u] = *reinterpret_cast<const float4*>(src);
-              v1[u] = *reinterpret_cast<const float4*>(src + 4);
-              wgt[u] = (l == -INFINITY) ? 0.f : expf(l - lse_all);
+        for (int u = 0; u < kPieceBatch; ++u) {
+          const int s = s0 + u;
+          lv[u] = -INFINITY;
+          v0[u] = v1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (s < np) {
+            const size_t pr = (size_t)(pb + s) * rows_total + row;
+            lv[u] = a.part_lse[pr];
+            if (cols) {
+              const float* src = a.part_o + pr * a.d_c + col0 + c0;
+              v0[u] = __ldcs(reinterpret_cast<const float4*>(src));
+              v1[u] = __ldcs(reinterpret_cast<const float4*>(src + 4));
             }
           }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            acc[0] += wgt[u] * v0[u].x; acc[1] += wgt[u] * v0[u].y;
-            acc[2] += wgt[u] * v0[u].z; acc[3] += wgt[u] * v0[u].w;
-            acc[4] += wgt[u] * v1[u].x; acc[5] += wgt[u] * v1[u].y;
-            acc[6] += wgt[u] * v1[u].z; acc[7] += wgt[u] * v1[u].w;
-          }
         }
-      }
-      uint32_t hi[4], lo[4];
+        float mb = m;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float x0 = acc[2 * e], x1 = acc[2 * e + 1];
-        hi[e] = pack_bf16x2(x0, x1);
-        lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+        for (int u = 0; u < kPieceBatch; ++u) mb = fmaxf(mb, lv[u]);
+        if (mb == -INFINITY) continue;                // nothing attended so far
+        const float sc = (m == -INFINITY) ? 0.f : expf(m - mb);
+        tot *= sc;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= sc;
+#pragma unroll
+        for (int u = 0; u < kPieceBatch; ++u) {
+          const float wu = (lv[u] == -INFINITY) ? 0.f : expf(lv[u] - mb);
+          tot += wu;
+          acc[0] += wu * v0[u].x; acc[1] += wu * v0[u].y;
+          acc[2] += wu * v0[u].z; acc[3] += wu * v0[u].w;
+          acc[4] += wu * v1[u].x; acc[5] += wu * v1[u].y;
+          acc[6] += wu * v1[u].z; acc[7] += wu * v1[u].w;
+        }
+        m = mb;
       }
-      *reinterpret_cast<uint4*>(o_hi + j * ostride + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(o_lo + j * ostride + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      const float lse_all = (m == -INFINITY) ? -INFINITY : m + logf(tot);
+      const float inv = (m == -INFINITY) ? 0.f : 1.f / tot;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] *= inv;
+      if (ks == 0 && gc == 0 && a.lse != nullptr) a.lse[(size_t)t * a.n_heads + h] = lse_all;
     }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = acc[2 * e], x1 = acc[2 * e + 1];
+      hi[e] = pack_bf16x2(x0, x1);
+      lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+    }
+    *reinterpret_cast<uint4*>(o_hi + j * kOStride + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(o_lo + j * kOStride + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
   __syncthreads();
 
-  // 2. out[t][v] = sum_c W_UV,h[v][c] o_lat[t][c]: warp per 16 value rows,
-  //    two 8-token tiles, reduction in 32-wide slices (see mma_frag.cuh)
-  const int g = lane >> 2, q = lane & 3;
-  const uint16_t* wh = a.w_uv + (size_t)h * a.v_head * a.d_c;
-  for (int m0 = warp * 16; m0 < a.v_head; m0 += 8 * 16) {
-    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-    const int va = m0 + g, vb = m0 + g + 8;
-    for (int kb = 0; kb < kpad; kb += 128) {          // four 32-wide slices' weights in flight at once
-      uint4 ra[4], rb[4];
-      const uint4 z = make_uint4(0, 0, 0, 0);
+  // 2. per chunk of 128 out rows: this slice's product (warp per 16 rows, two
+  //    8-token tiles, 32-wide k slices, see mma_frag.cuh), then the sum over
+  //    the cluster's KS slices
+  const uint32_t red_s = smem_addr(red);
+  for (int v0 = 0; v0 < a.v_head; v0 += kVChunk) {
+    if (v0 > 0) load_w(v0);
+    {
+      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int kk = kb + 32 * u + 8 * q;
-        const bool kin = kk < a.d_c;
-        ra[u] = (kin && va < a.v_head) ? ld_nc_v4(wh + (size_t)va * a.d_c + kk) : z;
-        rb[u] = (kin && vb < a.v_head) ? ld_nc_v4(wh + (size_t)vb * a.d_c + kk) : z;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int kk = kb + 32 * u + 8 * q;
-        if (kk >= kpad) break;
-        const uint4 h0 = *reinterpret_cast<const uint4*>(o_hi + g * ostride + kk);
-        const uint4 l0 = *reinterpret_cast<const uint4*>(o_lo + g * ostride + kk);
-        const uint4 h1 = *reinterpret_cast<const uint4*>(o_hi + (g + 8) * ostride + kk);
-        const uint4 l1 = *reinterpret_cast<const uint4*>(o_lo + (g + 8) * ostride + kk);
+        const int kk = 32 * u + 8 * q;
+        if (32 * u >= ncol) break;
+        const uint4 h0 = *reinterpret_cast<const uint4*>(o_hi + g * kOStride + kk);
+        const uint4 l0 = *reinterpret_cast<const uint4*>(o_lo + g * kOStride + kk);
+        const uint4 h1 = *reinterpret_cast<const uint4*>(o_hi + (g + 8) * kOStride + kk);
+        const uint4 l1 = *reinterpret_cast<const uint4*>(o_lo + (g + 8) * kOStride + kk);
         mma_k32(d0, ra[u], rb[u], h0);
         mma_k32(d0, ra[u], rb[u], l0);
         mma_k32(d1, ra[u], rb[u], h1);
         mma_k32(d1, ra[u], rb[u], l1);
       }
+      // D fragment: (row g | g+8, token column 2q | 2q+1) of each 8-token tile
+      const float* dd[2] = {d0, d1};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int vl = warp * 16 + g + ((e & 2) ? 8 : 0);
+          const int tl = nt * 8 + 2 * q + (e & 1);
+          red[vl * kTok + tl] = dd[nt][e];
+        }
     }
-    // D fragment: (row g | g+8, token column 2q | 2q+1) of each 8-token tile
-    const float* dd[2] = {d0, d1};
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int v = m0 + g + ((e & 2) ? 8 : 0);
-        const int t = t0 + nt * 8 + 2 * q + (e & 1);
-        if (v < a.v_head && t < T) a.out[((size_t)t * a.n_heads + h) * a.v_head + v] = f32_to_bf16(dd[nt][e]);
+    cluster_barrier();   // every slice's product of this chunk is in its CTA's shared memory
+    {
+      const int per = (kVChunk + KS - 1) / KS;    // rows of the chunk this CTA finishes
+      const int r0 = ks * per;
+      for (int idx = tid; idx < per * kTok; idx += kThreads) {
+        const int vl = r0 + idx / kTok, tl = idx % kTok;
+        const int v = v0 + vl, t = t0 + tl;
+        if (vl >= kVChunk || v >= a.v_head || t >= T) continue;
+        float sum = 0.f;
+        for (int r = 0; r < KS; ++r) sum += ld_cluster_f32(red_s + (uint32_t)(vl * kTok + tl) * 4u, (uint32_t)r);
+        a.out[((size_t)t * a.n_heads + h) * a.v_head + v] = f32_to_bf16(sum);
       }
     }
+    cluster_barrier();   // the peers have read this chunk before it is overwritten (or the CTA exits)
   }
 }
 
 }  // namespace
 
 size_t decode_combine_smem_bytes(int d_c) {
-  const int kpad = ((d_c + 31) & ~31);
-  return ((sizeof(PlanSmem) + 15) & ~size_t(15)) + 2ull * kTok * (kpad + 8) * 2;
+  (void)d_c;
+  return ((sizeof(PlanSmem) + 15) & ~size_t(15)) + 2ull * kTok * kOStride * 2 + (size_t)kVChunk * kTok * 4;
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
   const size_t smem = decode_combine_smem_bytes(a.d_c);
-  cudaError_t e = cudaFuncSetAttribute(decode_combine_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int T = a.batch * a.nq;
-  dim3 grid(a.n_heads, (T + kTok - 1) / kTok);
-  decode_combine_kernel<<<grid, kThreads, smem, stream>>>(a);
+  const int KS = (a.d_c + kSlice - 1) / kSlice;   // d_c <= 512: at most 4
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.n_heads, ((T + kTok - 1) / kTok) * KS, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = KS;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, a, KS);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -26,8 +26,7 @@
 // (bf16 pairs) [384, 512).
 //
 // Warp roles (320 threads): warp 0 lane 0 issues TMA loads (RoPE part of the
-// query tile once per piece, pages into a 4-stage ring, L2 prefetch further
-// ahead), warp 1 owns TMEM and lane 0 issues the MMAs, warps 2..5 (one per TMEM
+// query tile once per piece, pages into a 4-stage ring), warp 1 owns TMEM and lane 0 issues the MMAs, warps 2..5 (one per TMEM
 // lane quarter, one query row per thread) load the query tile's latent part into
 // TMEM and send the peer its partial scores, and warps 6..9 (same layout) run the
 // softmax and the epilogue.
@@ -51,7 +50,6 @@ using namespace sm100;
 
 constexpr int kThreads = 320;  // producer, MMA, 4 sender warps, 4 softmax warps
 constexpr int kStages = 4;
-constexpr int kPrefetch = 4;  // pages beyond the shared-memory ring prefetched into L2
 constexpr int kQrBytes = 128 * 64;            // RoPE block of the query tile [128 x 32] (64-byte swizzle)
 constexpr int kPageBytes = 4 * 8192 + 4096;   // 4 latent blocks [64 x 64] + RoPE block [64 x 32]
 constexpr int kXBytes = 128 * 64;             // received partial scores: [128 rows x 32 keys] fp16
@@ -235,19 +233,10 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // No L2 prefetch ahead of the ring: measured on this kernel and on a bare
+      // TMA stream of the same pages, prefetching slowed both (the prefetched
+      // lines compete with the ring's own loads and are partly evicted first).
       PageCursor cu(plan, a.batch, w);
-      // L2 prefetch runs kStages + kPrefetch pages ahead of the shared-memory loads;
-      // this CTA prefetches its 32 of the page's 64 rows (36 KB contiguous)
-      PageCursor pf(plan, a.batch, w);
-      bool more_pf = pf.next();
-      auto prefetch_next = [&]() {
-        if (!more_pf) return;
-        const int id = a.page_table[(size_t)pf.pc.b * a.max_pages + pf.pg];
-        if (id >= 0 && id < a.num_pages)
-          prefetch_l2(a.pool + ((size_t)id * 64 + 32 * c) * 576, 32 * 576 * 2);
-        more_pf = pf.next();
-      };
-      for (int i = 0; i < kStages + kPrefetch; ++i) prefetch_next();
       int issued[kStages] = {0, 0, 0, 0}, issued_q = 0;
       bool more = cu.next();
       int id_next = more ? a.page_table[(size_t)cu.pc.b * a.max_pages + cu.pg] : 0;
@@ -282,7 +271,6 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
         for (int i = 0; i < 4; ++i) tma_load_2d(dst + i * 8192, &tp128, c * 256 + 64 * i, id * 64, &bar->pg_full[st]);
         tma_load_2d(dst + 32768, &tp64, 512 + 32 * c, id * 64, &bar->pg_full[st]);
         ++issued[st];
-        prefetch_next();
       }
       if (*abort_flag) {
         // copies still in flight must land before this CTA's shared memory is released
