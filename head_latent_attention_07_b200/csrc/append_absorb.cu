@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(kAppWarps * 32)
 append_latent_kernel(AppendArgs a) {
   __shared__ float part[kAppWarps][16][17];
   __shared__ float red[kAppSplit][16][17];   // cluster leader: the split CTAs' tiles
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int R = a.d_c + a.d_rope;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, q = lane & 3;
@@ -113,6 +115,7 @@ append_latent_kernel(AppendArgs a) {
 
 // ------------------------------------------------------------------ absorb
 constexpr int kAbsThreads = 256;
+constexpr int kAbsMaxKSteps = 12;   // tensor-core path: qk_nope <= 192
 
 // RoPE(q_rope, pos) of one head for up to kTokBlk tokens.
 __device__ __forceinline__ void absorb_rope_part(const AbsorbArgs& a, int h, int t0) {
@@ -145,6 +148,8 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
 __global__ void __launch_bounds__(kAbsThreads)
 absorb_q_mma_kernel(AbsorbArgs a) {
   extern __shared__ __align__(16) uint16_t wsm[];   // [qk_nope][d_c + 8]
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int h = blockIdx.x;
   const int t0 = blockIdx.y * kTokBlk;
   const int dq = a.qk_nope + a.d_rope;
@@ -162,23 +167,35 @@ absorb_q_mma_kernel(AbsorbArgs a) {
                  : "memory");
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
-  absorb_rope_part(a, h, t0);
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();
+  // A fragments (q_nope of this warp's 16 tokens) for every k step, loaded once
+  // while W_UK,h streams in
   const int ta = t0 + g, tb = t0 + g + 8;
   const uint16_t* qa = a.q + ((size_t)ta * a.n_heads + h) * dq;
   const uint16_t* qb = a.q + ((size_t)tb * a.n_heads + h) * dq;
   const bool va = ta < a.n_tokens, vb = tb < a.n_tokens;
+  const int nks = a.qk_nope / 16;
+  uint32_t af[kAbsMaxKSteps][4];
+#pragma unroll
+  for (int k = 0; k < kAbsMaxKSteps; ++k) {
+    const int ia = 16 * k + 2 * q4;
+    const bool kin = k < nks;
+    af[k][0] = (kin && va) ? *reinterpret_cast<const uint32_t*>(qa + ia) : 0u;
+    af[k][1] = (kin && vb) ? *reinterpret_cast<const uint32_t*>(qb + ia) : 0u;
+    af[k][2] = (kin && va) ? *reinterpret_cast<const uint32_t*>(qa + ia + 8) : 0u;
+    af[k][3] = (kin && vb) ? *reinterpret_cast<const uint32_t*>(qb + ia + 8) : 0u;
+  }
+  absorb_rope_part(a, h, t0);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
   const int ntiles = a.d_c / 8;
   for (int nt0 = warp * 2; nt0 < ntiles; nt0 += 16) {  // pairs of 8-column tiles
     float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     const int j0 = nt0 * 8;
-    for (int i0 = 0; i0 < a.qk_nope; i0 += 16) {
-      const int ia = i0 + 2 * q4;
-      const uint32_t a0 = va ? *reinterpret_cast<const uint32_t*>(qa + ia) : 0u;
-      const uint32_t a1 = vb ? *reinterpret_cast<const uint32_t*>(qb + ia) : 0u;
-      const uint32_t a2 = va ? *reinterpret_cast<const uint32_t*>(qa + ia + 8) : 0u;
-      const uint32_t a3 = vb ? *reinterpret_cast<const uint32_t*>(qb + ia + 8) : 0u;
+#pragma unroll
+    for (int k = 0; k < kAbsMaxKSteps; ++k) {
+      if (k >= nks) break;
+      const int i0 = 16 * k;
+      const uint32_t a0 = af[k][0], a1 = af[k][1], a2 = af[k][2], a3 = af[k][3];
       // tiles: 0 = W[i0..+8][j0..+8], 1 = W[i0+8..][j0..], 2 = W[i0..][j0+8..], 3 = W[i0+8..][j0+8..]
       const int tile = lane >> 3, rr = lane & 7;
       const int wi = i0 + rr + ((tile & 1) ? 8 : 0);
@@ -202,6 +219,8 @@ absorb_q_mma_kernel(AbsorbArgs a) {
 __global__ void __launch_bounds__(kAbsThreads)
 absorb_q_kernel(AbsorbArgs a) {
   extern __shared__ __align__(16) float qn[];   // [kTokBlk][qk_nope]
+  allow_dependent_launch();
+  grid_dependency_wait();
   const int h = blockIdx.x;
   const int t0 = blockIdx.y * kTokBlk;
   const int dq = a.qk_nope + a.d_rope;
@@ -247,13 +266,14 @@ cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream) {
   cfg.gridDim = dim3((R + 15) / 16, (a.n_tokens + kTokBlk - 1) / kTokBlk, kAppSplit);
   cfg.blockDim = dim3(kAppWarps * 32, 1, 1);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = kAppSplit;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, append_latent_kernel, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -262,11 +282,20 @@ cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream) {
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream) {
   dim3 grid(a.n_heads, (a.n_tokens + kTokBlk - 1) / kTokBlk);
   const size_t wsmem = (size_t)a.qk_nope * (a.d_c + 8) * 2;
-  if (a.qk_nope % 16 == 0 && a.d_c % 8 == 0 && wsmem <= 200 * 1024) {
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kAbsThreads, 1, 1);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.qk_nope % 16 == 0 && a.qk_nope <= 16 * kAbsMaxKSteps && a.d_c % 8 == 0 && wsmem <= 200 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(absorb_q_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)wsmem);
     if (e != cudaSuccess) return e;
-    absorb_q_mma_kernel<<<grid, kAbsThreads, wsmem, stream>>>(a);
+    cfg.dynamicSmemBytes = wsmem;
+    e = cudaLaunchKernelEx(&cfg, absorb_q_mma_kernel, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
   const size_t smem = (size_t)kTokBlk * a.qk_nope * 4;
@@ -274,7 +303,9 @@ cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(absorb_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  absorb_q_kernel<<<grid, kAbsThreads, smem, stream>>>(a);
+  cfg.dynamicSmemBytes = smem;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, absorb_q_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -45,15 +45,22 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 // ---------------------------------------------------------------- RoPE
 // Rotation of channel pair (2i, 2i+1) of a width-d RoPE vector at position pos:
 // angle = pos * theta^(-2i/d), evaluated in double precision so that positions
-// up to 2^31 keep their phase; the cosine/sine are rounded to fp32.
+// up to 2^31 keep their phase, then reduced modulo 2 pi in double precision; the
+// cosine and sine of the remainder (|r| <= pi) are taken in fp32.
 __device__ __forceinline__ void rope_cos_sin(int pos, int i, int d, float theta, float* c, float* s) {
-  double inv_freq = pow((double)theta, -2.0 * (double)i / (double)d);
-  double ang = (double)pos * inv_freq;
-  double sd, cd;
-  sincos(ang, &sd, &cd);
-  *c = (float)cd;
-  *s = (float)sd;
+  const double inv_freq = pow((double)theta, -2.0 * (double)i / (double)d);
+  const double ang = (double)pos * inv_freq;
+  const double two_pi = 6.283185307179586476925286766559;
+  const double k = rint(ang * (1.0 / two_pi));
+  const float r = (float)fma(-k, two_pi, ang);
+  sincosf(r, s, c);
 }
+
+// Programmatic dependent launch: the next kernel on the stream may start its
+// prologue early; every kernel waits for its predecessor's completion (and the
+// visibility of its writes) before it reads any input.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

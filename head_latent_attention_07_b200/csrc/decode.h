@@ -54,6 +54,16 @@ bool decode_tc_supported(int d_c, int d_rope, int page_size);
 int decode_tc_workers(int sms, int rows_total);
 cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cudaStream_t stream);
 constexpr long long kSpinLimitCycles = 1ll << 31;  // ~1 s at B200 clocks per bounded wait
+
+// Launch attribute that lets a kernel start while its predecessor on the stream
+// finishes (every kernel of this library waits for the predecessor, with
+// griddepcontrol.wait, before it reads any input).
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
+  return at;
+}
 cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
 

@@ -57,6 +57,8 @@ decode_combine_kernel(DecodeArgs a, int KS) {
   uint16_t* o_lo = o_hi + kTok * kOStride;
   float* red = reinterpret_cast<float*>(o_lo + kTok * kOStride);   // [kVChunk][kTok] partial products
 
+  allow_dependent_launch();
+  grid_dependency_wait();   // the partials of the split kernel
   build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr);
   const int h = blockIdx.x;
   const int ks = (int)cta_rank();
@@ -224,13 +226,14 @@ cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = KS;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, a, KS);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -37,6 +37,8 @@ decode_split_simt_kernel(DecodeArgs a) {
   uint16_t* page_s = reinterpret_cast<uint16_t*>(q_s + kRows * R);                           // [P][R]
   float* s_s = reinterpret_cast<float*>(page_s + a.page_size * R);                            // [kRows][P]
 
+  allow_dependent_launch();
+  grid_dependency_wait();
   build_plan(&sm->plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.dev_status);
   const int w = blockIdx.x;
   const int row0 = blockIdx.y * kRows;
@@ -219,8 +221,16 @@ cudaError_t launch_decode_split_simt(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(decode_split_simt_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.G, decode_simt_row_groups(a.nq * a.n_heads));
-  decode_split_simt_kernel<<<grid, kThreads, smem, stream>>>(a);
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.G, decode_simt_row_groups(a.nq * a.n_heads));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_split_simt_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

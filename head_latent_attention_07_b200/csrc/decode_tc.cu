@@ -223,6 +223,9 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
   }
+  // setup above touches no input: the predecessor on the stream may still run
+  allow_dependent_launch();
+  grid_dependency_wait();
   build_plan(plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G,
              (blockIdx.x == 0 && blockIdx.y == 0) ? status : nullptr);  // ends with __syncthreads
   tc_fence_before();
@@ -714,13 +717,14 @@ cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cu
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, decode_split_tc_kernel, tq64, tp128, tp64, prm);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
