@@ -93,7 +93,8 @@ int mla_append_latent(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w
   a.h = h; a.w_dkv = w_dkv; a.seq_idx = seq_idx; a.pos = pos; a.page_table = page_table;
   a.pool = pool; a.dev_status = dev_status; a.n_tokens = n_tokens; a.d_model = dims->d_model;
   a.d_c = dims->d_c; a.d_rope = dims->d_rope; a.page_size = dims->page_size; a.batch = batch;
-  a.max_pages = max_pages; a.num_pages = num_pages; a.theta = eff_theta(dims);
+  a.max_pages = max_pages; a.num_pages = num_pages;
+  mla::rope_inv_freq(a.inv_freq, dims->d_rope, eff_theta(dims));
   return cuda_status(mla::launch_append_latent(a, (cudaStream_t)stream));
 }
 
@@ -108,7 +109,7 @@ int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
   mla::AbsorbArgs a;
   a.q = q; a.pos = pos; a.w_uk = w_uk; a.q_lat = q_lat; a.n_tokens = n_tokens;
   a.n_heads = dims->n_heads; a.qk_nope = dims->qk_nope; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
-  a.theta = eff_theta(dims);
+  mla::rope_inv_freq(a.inv_freq, dims->d_rope, eff_theta(dims));
   return cuda_status(mla::launch_absorb_q(a, (cudaStream_t)stream));
 }
 

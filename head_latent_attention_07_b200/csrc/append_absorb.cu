@@ -22,7 +22,7 @@ constexpr int kTokBlk = 16;
 // in 32-wide slices (mma_frag.cuh), their partial tiles are summed in shared
 // memory, then RoPE is applied to the k^ rows and the bf16 row goes to its slot.
 constexpr int kAppWarps = 8;
-constexpr int kAppSplit = 4;   // CTAs of a cluster splitting the reduction over D
+constexpr int kAppSplit = 8;   // CTAs of a cluster splitting the reduction over D
 
 __global__ void __launch_bounds__(kAppWarps * 32)
 append_latent_kernel(AppendArgs a) {
@@ -85,7 +85,10 @@ append_latent_kernel(AppendArgs a) {
   __shared__ float vals[16][17];
   {
     const int row = threadIdx.x >> 4, tok = threadIdx.x & 15;
-    vals[row][tok] = (red[0][row][tok] + red[1][row][tok]) + (red[2][row][tok] + red[3][row][tok]);
+    float v = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < kAppSplit; ++sp) v += red[sp][row][tok];
+    vals[row][tok] = v;
   }
   __syncthreads();
   // store: thread (row, token); RoPE rows pair up inside the tile (m0 and d_c are even)
@@ -106,7 +109,7 @@ append_latent_kernel(AppendArgs a) {
   if (row >= a.d_c) {
     const int qch = row - a.d_c;          // channel within the RoPE key
     float c, s;
-    rope_cos_sin(p, qch >> 1, a.d_rope, a.theta, &c, &s);
+    rope_cos_sin(p, a.inv_freq[qch >> 1], &c, &s);
     const float x0 = vals[rr & ~1][j], x1 = vals[rr | 1][j];
     val = (qch & 1) ? x0 * s + x1 * c : x0 * c - x1 * s;
   }
@@ -129,7 +132,7 @@ __device__ __forceinline__ void absorb_rope_part(const AbsorbArgs& a, int h, int
     const uint16_t* src = a.q + ((size_t)t * a.n_heads + h) * dq + a.qk_nope + 2 * i;
     const float x0 = bf16_to_f32(src[0]), x1 = bf16_to_f32(src[1]);
     float c, s;
-    rope_cos_sin(a.pos[t], i, a.d_rope, a.theta, &c, &s);
+    rope_cos_sin(a.pos[t], a.inv_freq[i], &c, &s);
     *reinterpret_cast<uint32_t*>(a.q_lat + ((size_t)t * a.n_heads + h) * R + a.d_c + 2 * i) =
         pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
   }

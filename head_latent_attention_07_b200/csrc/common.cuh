@@ -43,12 +43,11 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 }
 
 // ---------------------------------------------------------------- RoPE
-// Rotation of channel pair (2i, 2i+1) of a width-d RoPE vector at position pos:
-// angle = pos * theta^(-2i/d), evaluated in double precision so that positions
-// up to 2^31 keep their phase, then reduced modulo 2 pi in double precision; the
-// cosine and sine of the remainder (|r| <= pi) are taken in fp32.
-__device__ __forceinline__ void rope_cos_sin(int pos, int i, int d, float theta, float* c, float* s) {
-  const double inv_freq = pow((double)theta, -2.0 * (double)i / (double)d);
+// Rotation of a RoPE channel pair at position pos, inv_freq = theta^(-2i/d) of
+// the pair: the angle pos * inv_freq is evaluated in double precision so that
+// positions up to 2^31 keep their phase, then reduced modulo 2 pi in double
+// precision; the cosine and sine of the remainder (|r| <= pi) are taken in fp32.
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
   const double ang = (double)pos * inv_freq;
   const double two_pi = 6.283185307179586476925286766559;
   const double k = rint(ang * (1.0 / two_pi));

@@ -7,6 +7,13 @@
 
 namespace mla {
 
+constexpr int kMaxRopePairs = 128;  // d_rope <= 256
+
+// theta^(-2i/d_rope) for the RoPE channel pairs (host side, double precision).
+inline void rope_inv_freq(double* out, int d_rope, float theta) {
+  for (int i = 0; i < d_rope / 2 && i < kMaxRopePairs; ++i) out[i] = pow((double)theta, -2.0 * i / d_rope);
+}
+
 struct DecodeArgs {
   const uint16_t* q_lat;      // [B, nq, H, R]
   const uint16_t* pool;       // [num_pages, P, R]
@@ -32,7 +39,7 @@ struct AppendArgs {
   uint16_t* pool;             // [num_pages, P, R]
   int32_t* dev_status;
   int n_tokens, d_model, d_c, d_rope, page_size, batch, max_pages, num_pages;
-  float theta;
+  double inv_freq[kMaxRopePairs];   // theta^(-2i/d_rope), computed on the host in double precision
 };
 
 struct AbsorbArgs {
@@ -41,7 +48,7 @@ struct AbsorbArgs {
   const uint16_t* w_uk;       // [H, d_n, d_c]
   uint16_t* q_lat;            // [T, H, d_c + d_r]
   int n_tokens, n_heads, qk_nope, d_c, d_rope;
-  float theta;
+  double inv_freq[kMaxRopePairs];
 };
 
 size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);
