@@ -57,8 +57,11 @@ decode_combine_kernel(DecodeArgs a, int KS) {
   uint16_t* o_lo = o_hi + kTok * kOStride;
   float* red = reinterpret_cast<float*>(o_lo + kTok * kOStride);   // [kVChunk][kTok] partial products
 
+  // The predecessor on the stream is always this call's split kernel, which
+  // writes only the partials and lets this kernel launch only after its own
+  // dependency wait: seq_lens and W_UV are final here, the partials after the
+  // wait below.
   allow_dependent_launch();
-  grid_dependency_wait();   // the partials of the split kernel
   build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr);
   const int h = blockIdx.x;
   const int ks = (int)cta_rank();
@@ -86,6 +89,7 @@ decode_combine_kernel(DecodeArgs a, int KS) {
     }
   };
   load_w(0);
+  grid_dependency_wait();   // the split kernel's partials
 
   // 1. merge: 16 threads per token, each owning 8 consecutive columns of the
   //    slice; one pass over the pieces in batches of 8 (their LSEs and partial

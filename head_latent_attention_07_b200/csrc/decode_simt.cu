@@ -37,8 +37,8 @@ decode_split_simt_kernel(DecodeArgs a) {
   uint16_t* page_s = reinterpret_cast<uint16_t*>(q_s + kRows * R);                           // [P][R]
   float* s_s = reinterpret_cast<float*>(page_s + a.page_size * R);                            // [kRows][P]
 
-  allow_dependent_launch();
   grid_dependency_wait();
+  allow_dependent_launch();   // after the wait: see decode_tc.cu
   build_plan(&sm->plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.dev_status);
   const int w = blockIdx.x;
   const int row0 = blockIdx.y * kRows;

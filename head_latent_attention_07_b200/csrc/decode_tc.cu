@@ -224,8 +224,10 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
     tmem_relinquish();
   }
   // setup above touches no input: the predecessor on the stream may still run
-  allow_dependent_launch();
   grid_dependency_wait();
+  // only now may the combine launch: its prologue reads seq_lens and W_UV,
+  // whose producers (if any) ran before this kernel's wait returned
+  allow_dependent_launch();
   build_plan(plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G,
              (blockIdx.x == 0 && blockIdx.y == 0) ? status : nullptr);  // ends with __syncthreads
   tc_fence_before();
