@@ -101,6 +101,23 @@ def profiled_traffic(workload_name: str):
     return int(fields["traffic_bytes_per_call"]), "ncu dram__bytes_read.sum + dram__bytes_write.sum, split + combine"
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (all ranks get the result); the
+    identity when no process group is running."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch of tokens_per_rank
+    query tokens per step (weak scaling), timed by the slowest rank."""
+    return world * tokens_per_rank * steps / (ms / 1000.0)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -288,11 +305,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
     # the copies really happened: the last output read back equals the device result
     assert torch.equal(out_host[(args.steps - 1) % 2], outs[(args.steps - 1) % 2].cpu()), "e2e output copy"
 
-    times = torch.tensor([ms_total, e2e_ms, float(np.mean(decode_ms))], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms, dec_ms = times.tolist()
+    ms_total, e2e_ms, dec_ms = max_over_ranks([ms_total, e2e_ms, float(np.mean(decode_ms))], dev)
     return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": dec_ms, "clocks": clocks,
             "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens}
 
@@ -405,7 +418,7 @@ def main():
     peaks, src = load_peaks()
     cnt = algorithmic_counts(w, r["lens"])
     T = w.tokens
-    value = world * T * args.steps / (r["ms_total"] / 1000.0)
+    value = job_throughput(world, T, args.steps, r["ms_total"])
     dec_s = r["decode_ms"] / 1000.0
     gbs = cnt["bytes"] / dec_s / 1e9
     tfs = cnt["flops"] / dec_s / 1e12
@@ -429,7 +442,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**describe(w), "parallelism": f"dp{world} (independent replicas)"},
             "roofline": roof,
-            "e2e": {"value": world * T * args.steps / (r["e2e_ms"] / 1000.0), "unit": "tokens/s",
+            "e2e": {"value": job_throughput(world, T, args.steps, r["e2e_ms"]), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                     "copies": "pinned host buffers, double-buffered on a second stream, inside the timed region"},
             "gpu_launches": r["launches"], "clocks": r["clocks"]}
