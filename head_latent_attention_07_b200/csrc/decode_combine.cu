@@ -5,15 +5,16 @@
 //   o_lat = sum_s exp(lse_s - LSE) * O_s          (O_s already normalised per piece)
 //   out[t][h][v] = sum_c W_UV[h][v][c] * o_lat[c]  (values up-projected once, after
 //                                                   attending over latents)
-// Work split: a cluster of KS = ceil(d_c / 128) CTAs per (head, group of 16
-// query tokens); CTA ks owns latent columns [128 ks, 128 ks + 128).  It merges
+// Work split: a cluster of KS = ceil(d_c / 256) CTAs per (head, group of 16
+// query tokens); CTA ks owns latent columns [256 ks, 256 ks + 256).  It merges
 // its columns of the partials (each partial byte is read once, by one CTA) and
-// multiplies them by its 128-column slice of W_UV,h on the tensor cores
+// multiplies them by its 256-column slice of W_UV,h on the tensor cores
 // (mma.sync, fp32 accumulate, o_lat split into two bf16 terms, hi + lo, which
-// keeps about 16 bits of its mantissa).  The KS partial products are summed
+// keeps about 16 bits of its mantissa).  The KS slice products are summed
 // through distributed shared memory, each CTA finishing 1/KS of the rows of
-// out.  Many small CTAs keep enough loads in flight to stream the partials and
-// W_UV at memory speed.
+// out.  At d_c = 512 and 16 query tokens this is 2 CTAs per head, all resident
+// at once (one wave at two CTAs per SM); the W_UV slice streams into shared
+// memory before the kernel waits for the split kernel's partials.
 #include "common.cuh"
 #include "decode.h"
 #include "mma_frag.cuh"
@@ -25,10 +26,11 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTok = 16;       // query tokens per CTA
-constexpr int kSlice = 128;    // latent columns per CTA
-constexpr int kVChunk = 128;   // out rows reduced per cluster round
+constexpr int kSlice = 256;    // latent columns per CTA
+constexpr int kVChunk = 128;   // out rows per round (8 warps x 16)
 constexpr int kOStride = kSlice + 8;   // bf16 row stride of the merged slice (16-byte pad)
-constexpr int kPieceBatch = 6;         // pieces whose loads are in flight at once
+constexpr int kWStride = kSlice + 8;   // bf16 row stride of the staged W_UV slice (16-byte pad)
+constexpr int kPieceBatch = 4;         // pieces whose loads are in flight at once
 
 __device__ __forceinline__ uint32_t cta_rank() {
   uint32_t r;
@@ -55,14 +57,9 @@ decode_combine_kernel(DecodeArgs a, int KS) {
   PlanSmem* ps = reinterpret_cast<PlanSmem*>(smem_raw);
   uint16_t* o_hi = reinterpret_cast<uint16_t*>(smem_raw + ((sizeof(PlanSmem) + 15) & ~size_t(15)));
   uint16_t* o_lo = o_hi + kTok * kOStride;
-  float* red = reinterpret_cast<float*>(o_lo + kTok * kOStride);   // [kVChunk][kTok] partial products
+  float* red = reinterpret_cast<float*>(o_lo + kTok * kOStride);       // [kVChunk][kTok] slice products
+  uint16_t* wsm = reinterpret_cast<uint16_t*>(red + kVChunk * kTok);  // [kVChunk][kWStride] W_UV slice
 
-  // The predecessor on the stream is always this call's split kernel, which
-  // writes only the partials and lets this kernel launch only after its own
-  // dependency wait: seq_lens and W_UV are final here, the partials after the
-  // wait below.
-  allow_dependent_launch();
-  build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr);
   const int h = blockIdx.x;
   const int ks = (int)cta_rank();
   const int t0 = (blockIdx.y / KS) * kTok;
@@ -71,58 +68,71 @@ decode_combine_kernel(DecodeArgs a, int KS) {
   const int col0 = ks * kSlice;
   const int ncol = min(kSlice, a.d_c - col0);   // multiple of 8
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  // this slice's weights for the first chunk of out rows, loaded before the
-  // merge so that their latency overlaps it (see step 2 for the fragment layout)
   const int g = lane >> 2, q = lane & 3;
   const uint16_t* wh = a.w_uv + (size_t)h * a.v_head * a.d_c + col0;
-  uint4 ra[4], rb[4];
-  auto load_w = [&](int v0) {
-    const int va = v0 + warp * 16 + g, vb = va + 8;
-    const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {                   // four 32-wide k slices in flight
-      const int kk = 32 * u + 8 * q;
-      const bool kin = kk < ncol;
-      ra[u] = (kin && va < a.v_head) ? ldg_stream(wh + (size_t)va * a.d_c + kk) : z;
-      rb[u] = (kin && vb < a.v_head) ? ldg_stream(wh + (size_t)vb * a.d_c + kk) : z;
+  // this slice of W_UV,h for a chunk of out rows -> shared memory (zeros outside it)
+  auto stage_w = [&](int v0) {
+    for (int idx = tid; idx < kVChunk * (kSlice / 8); idx += kThreads) {
+      const int vl = idx / (kSlice / 8), cc = 8 * (idx % (kSlice / 8));
+      uint16_t* dst = wsm + vl * kWStride + cc;
+      if (v0 + vl < a.v_head && cc < ncol) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)),
+                     "l"(wh + (size_t)(v0 + vl) * a.d_c + cc)
+                     : "memory");
+      } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  load_w(0);
+
+  // The predecessor on the stream is always this call's split kernel, which
+  // writes only the partials and lets this kernel launch only after its own
+  // dependency wait: seq_lens and W_UV are final here, the partials after the
+  // wait below.
+  allow_dependent_launch();
+  stage_w(0);
+  build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr);
   grid_dependency_wait();   // the split kernel's partials
 
-  // 1. merge: 16 threads per token, each owning 8 consecutive columns of the
-  //    slice; one pass over the pieces in batches of 8 (their LSEs and partial
-  //    rows loaded together), with the running max moved as batches arrive
+  // 1. merge: 16 threads per token, each owning columns [8 gc, 8 gc + 8) and
+  //    [128 + 8 gc, 128 + 8 gc + 8) of the slice; one pass over the pieces in
+  //    batches (their LSEs and partial rows loaded together), with the running
+  //    max moved as batches arrive
   {
     const int j = tid >> 4, gc = tid & 15;
     const int t = t0 + j;
-    const int c0 = 8 * gc;
-    float acc[8];
+    float acc[16];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
     if (t < T) {
       const int b = t / a.nq, i = t % a.nq;
       const int row = i * a.n_heads + h;
       const int pb = ps->piece_begin[b];
       const int np = ps->piece_begin[b + 1] - pb;
-      const bool cols = c0 < ncol;
+      bool cols[2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) cols[half] = 128 * half + 8 * gc < ncol;
       float m = -INFINITY, tot = 0.f;
       for (int s0 = 0; s0 < np; s0 += kPieceBatch) {
         float lv[kPieceBatch];
-        float4 v0[kPieceBatch], v1[kPieceBatch];
+        float4 v[kPieceBatch][4];
 #pragma unroll
         for (int u = 0; u < kPieceBatch; ++u) {
           const int s = s0 + u;
           lv[u] = -INFINITY;
-          v0[u] = v1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) v[u][k] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (s < np) {
             const size_t pr = (size_t)(pb + s) * rows_total + row;
             lv[u] = a.part_lse[pr];
-            if (cols) {
-              const float* src = a.part_o + pr * a.d_c + col0 + c0;
-              v0[u] = __ldcs(reinterpret_cast<const float4*>(src));
-              v1[u] = __ldcs(reinterpret_cast<const float4*>(src + 4));
+            const float* src = a.part_o + pr * a.d_c + col0 + 8 * gc;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              if (cols[half]) {
+                v[u][2 * half] = __ldcs(reinterpret_cast<const float4*>(src + 128 * half));
+                v[u][2 * half + 1] = __ldcs(reinterpret_cast<const float4*>(src + 128 * half + 4));
+              }
             }
           }
         }
@@ -133,34 +143,42 @@ decode_combine_kernel(DecodeArgs a, int KS) {
         const float sc = (m == -INFINITY) ? 0.f : expf(m - mb);
         tot *= sc;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] *= sc;
+        for (int e = 0; e < 16; ++e) acc[e] *= sc;
 #pragma unroll
         for (int u = 0; u < kPieceBatch; ++u) {
           const float wu = (lv[u] == -INFINITY) ? 0.f : expf(lv[u] - mb);
           tot += wu;
-          acc[0] += wu * v0[u].x; acc[1] += wu * v0[u].y;
-          acc[2] += wu * v0[u].z; acc[3] += wu * v0[u].w;
-          acc[4] += wu * v1[u].x; acc[5] += wu * v1[u].y;
-          acc[6] += wu * v1[u].z; acc[7] += wu * v1[u].w;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            acc[4 * k + 0] += wu * v[u][k].x;
+            acc[4 * k + 1] += wu * v[u][k].y;
+            acc[4 * k + 2] += wu * v[u][k].z;
+            acc[4 * k + 3] += wu * v[u][k].w;
+          }
         }
         m = mb;
       }
       const float lse_all = (m == -INFINITY) ? -INFINITY : m + logf(tot);
       const float inv = (m == -INFINITY) ? 0.f : 1.f / tot;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] *= inv;
+      for (int e = 0; e < 16; ++e) acc[e] *= inv;
       if (ks == 0 && gc == 0 && a.lse != nullptr) a.lse[(size_t)t * a.n_heads + h] = lse_all;
     }
-    uint32_t hi[4], lo[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float x0 = acc[2 * e], x1 = acc[2 * e + 1];
-      hi[e] = pack_bf16x2(x0, x1);
-      lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+    for (int half = 0; half < 2; ++half) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = acc[8 * half + 2 * e], x1 = acc[8 * half + 2 * e + 1];
+        hi[e] = pack_bf16x2(x0, x1);
+        lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
+      }
+      const int c0 = 128 * half + 8 * gc;
+      *reinterpret_cast<uint4*>(o_hi + j * kOStride + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(o_lo + j * kOStride + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    *reinterpret_cast<uint4*>(o_hi + j * kOStride + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(o_lo + j * kOStride + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
   // 2. per chunk of 128 out rows: this slice's product (warp per 16 rows, two
@@ -168,21 +186,28 @@ decode_combine_kernel(DecodeArgs a, int KS) {
   //    the cluster's KS slices
   const uint32_t red_s = smem_addr(red);
   for (int v0 = 0; v0 < a.v_head; v0 += kVChunk) {
-    if (v0 > 0) load_w(v0);
+    if (v0 > 0) {
+      stage_w(v0);
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();
+    }
     {
       float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      const int va = warp * 16 + g, vb = va + 8;
+#pragma unroll 2
+      for (int u = 0; u < kSlice / 32; ++u) {
         const int kk = 32 * u + 8 * q;
         if (32 * u >= ncol) break;
+        const uint4 wa = *reinterpret_cast<const uint4*>(wsm + va * kWStride + kk);
+        const uint4 wb = *reinterpret_cast<const uint4*>(wsm + vb * kWStride + kk);
         const uint4 h0 = *reinterpret_cast<const uint4*>(o_hi + g * kOStride + kk);
         const uint4 l0 = *reinterpret_cast<const uint4*>(o_lo + g * kOStride + kk);
         const uint4 h1 = *reinterpret_cast<const uint4*>(o_hi + (g + 8) * kOStride + kk);
         const uint4 l1 = *reinterpret_cast<const uint4*>(o_lo + (g + 8) * kOStride + kk);
-        mma_k32(d0, ra[u], rb[u], h0);
-        mma_k32(d0, ra[u], rb[u], l0);
-        mma_k32(d1, ra[u], rb[u], h1);
-        mma_k32(d1, ra[u], rb[u], l1);
+        mma_k32(d0, wa, wb, h0);
+        mma_k32(d0, wa, wb, l0);
+        mma_k32(d1, wa, wb, h1);
+        mma_k32(d1, wa, wb, l1);
       }
       // D fragment: (row g | g+8, token column 2q | 2q+1) of each 8-token tile
       const float* dd[2] = {d0, d1};
@@ -208,7 +233,7 @@ decode_combine_kernel(DecodeArgs a, int KS) {
         a.out[((size_t)t * a.n_heads + h) * a.v_head + v] = f32_to_bf16(sum);
       }
     }
-    cluster_barrier();   // the peers have read this chunk before it is overwritten (or the CTA exits)
+    cluster_barrier();   // the peers have read this chunk (and this CTA its W slice) before reuse or exit
   }
 }
 
@@ -216,7 +241,8 @@ decode_combine_kernel(DecodeArgs a, int KS) {
 
 size_t decode_combine_smem_bytes(int d_c) {
   (void)d_c;
-  return ((sizeof(PlanSmem) + 15) & ~size_t(15)) + 2ull * kTok * kOStride * 2 + (size_t)kVChunk * kTok * 4;
+  return ((sizeof(PlanSmem) + 15) & ~size_t(15)) + 2ull * kTok * kOStride * 2 + (size_t)kVChunk * kTok * 4 +
+         (size_t)kVChunk * kWStride * 2;
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
@@ -224,7 +250,7 @@ cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int T = a.batch * a.nq;
-  const int KS = (a.d_c + kSlice - 1) / kSlice;   // d_c <= 512: at most 4
+  const int KS = (a.d_c + kSlice - 1) / kSlice;   // d_c <= 512: at most 2
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.n_heads, ((T + kTok - 1) / kTok) * KS, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
