@@ -245,6 +245,27 @@ def attend_brute(q, q_pos, C, KR, w_uk, w_uv, scale, theta=DEFAULT_THETA):
 
 
 # ----------------------------------------------------------------------------
+# Layer output projection
+# ----------------------------------------------------------------------------
+
+def out_project(o: np.ndarray, w_o: np.ndarray) -> np.ndarray:
+    """Layer output y[t] = W_O concat_h(o[t, h]).
+
+    [distaisys] sec. 3: the attention output of every head is laid side by side,
+    head after head (input index h * d_v + j), and one bias-free linear map of
+    width H * d_v -> d_model produces the layer output.  [from-scratch]
+    "Absorption, and why RoPE breaks it": on the value side W_UV is applied once
+    after attending over the latents, right before this map, so the two fold into
+    one matrix by associativity.
+
+    o [T, H, d_v]; w_o [d_model, H * d_v] ([out, in]).  Returns y [T, d_model].
+    """
+    o = np.asarray(o, dtype=np.float64)
+    x = o.reshape(o.shape[0], o.shape[1] * o.shape[2])   # head-major concatenation
+    return x @ np.asarray(w_o, dtype=np.float64).T
+
+
+# ----------------------------------------------------------------------------
 # Split-KV partials and their log-sum-exp merge
 # ----------------------------------------------------------------------------
 
