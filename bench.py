@@ -20,6 +20,10 @@ positions, lengths) copied from pinned host memory and its output copied back,
 inside the timed region, double-buffered on a second stream the way a serving
 loop overlaps transfers with the neighbouring steps' compute.
 
+next_rows.out_proj: the layer output projection y = W_O concat_h(o_h)
+(mla_out_proj) on the step's output, timed alone after the step (it is not part
+of the step); W_O (235 MB at the V3 shape) is larger than L2.
+
 --impl reference times the CPU oracle (float64 numpy, absorbed form) on a
 bounded sample of the same workload on the host cores, as the comparison arm.
 """
@@ -305,9 +309,36 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
     # the copies really happened: the last output read back equals the device result
     assert torch.equal(out_host[(args.steps - 1) % 2], outs[(args.steps - 1) % 2].cpu()), "e2e output copy"
 
-    ms_total, e2e_ms, dec_ms = max_over_ranks([ms_total, e2e_ms, float(np.mean(decode_ms))], dev)
+    op = measure_out_proj(M, w, dims, out, dev, stream, args.seed + rank)
+
+    ms_total, e2e_ms, dec_ms, op_us = max_over_ranks(
+        [ms_total, e2e_ms, float(np.mean(decode_ms)), op["time_us"]], dev)
+    op["time_us"] = op_us
     return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": dec_ms, "clocks": clocks,
-            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens}
+            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens,
+            "out_proj": op}
+
+
+def measure_out_proj(M, w: W.Workload, dims, out, dev, stream, seed: int, iters: int = 50) -> dict:
+    """Average device time of mla_out_proj over `iters` back-to-back launches on
+    the decode output `out` (CUDA events on the launching stream, 3 warm-up launches)."""
+    import torch
+    x = W.make_out_proj_inputs(w, seed, w.tokens)
+    w_o = torch.from_numpy(x["w_o"]).view(torch.bfloat16).to(dev)
+    y = torch.empty((w.tokens, w.d_model), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        M.mla_out_proj(dims, out, w_o, y, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        M.mla_out_proj(dims, out, w_o, y, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    nbytes = (w_o.numel() + out.numel() + y.numel()) * 2
+    return {"time_us": e0.elapsed_time(e1) * 1000.0 / iters, "bytes_per_launch": nbytes, "launches": iters,
+            "tokens": w.tokens, "shape": f"y[{w.tokens}, {w.d_model}] = o[{w.tokens}, {w.n_heads * w.v_head}]"
+                                         f" . W_O[{w.d_model}, {w.n_heads * w.v_head}]^T"}
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -446,6 +477,13 @@ def main():
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                     "copies": "pinned host buffers, double-buffered on a second stream, inside the timed region"},
             "gpu_launches": r["launches"], "clocks": r["clocks"]}
+    op = r["out_proj"]
+    op_gbs = op["bytes_per_launch"] / (op["time_us"] * 1e-6) / 1e9
+    line["next_rows"] = {"out_proj": {
+        "kernel": "out_proj_kernel (mla_out_proj), timed alone after the step, not part of it",
+        "shape": op["shape"], "bound": "hbm", "achieved": op_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": op_gbs / peaks["hbm_gbs"], "time_us": op["time_us"], "bytes_per_launch": op["bytes_per_launch"],
+        "launches_timed": op["launches"], "l2": "W_O is larger than L2"}}
     if world == 1 and not args.no_cpu_baseline:
         arm = OracleArm(w, args.seed)
         v, sample = arm.measure(args.cpu_budget)

@@ -39,6 +39,7 @@ SIGNATURES = {
     "mla_decode_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, ctypes.c_size_t,
                                        _P, _P, _P, _P]),
     "mla_decode_attn_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "mla_out_proj": (ctypes.c_int, [_P, _P, _P, _P, _I, _P]),
     "mla_status_read": (ctypes.c_int, [_P, _P]),
     "mla_status_clear": (ctypes.c_int, [_P, _P]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -235,6 +236,21 @@ def mla_decode_attn_noalloc(dims: MlaDims, q_lat, pool, page_table, seq_lens, w_
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
         _ptr(dev_status, torch.int32, "dev_status"), _stream(stream))
     _check(st, "mla_decode_attn_noalloc")
+
+
+def mla_out_proj(dims: MlaDims, o, w_o, y, stream=None) -> None:
+    """Layer output y [T, d_model] = W_O concat_h(o[t, h]) for o [T, H, v_head]
+    (or the [B, nq, H, v_head] output of mla_decode_attn)."""
+    torch = _torch()
+    T = o.numel() // (dims.n_heads * dims.v_head) if o.dim() >= 2 else -1
+    if o.dim() < 3 or tuple(o.shape[-2:]) != (dims.n_heads, dims.v_head):
+        raise ValueError(f"o must be [..., {dims.n_heads}, {dims.v_head}], got {tuple(o.shape)}")
+    _shape(w_o, (dims.d_model, dims.n_heads * dims.v_head), "w_o")
+    _shape(y, (T, dims.d_model), "y")
+    st = load_library().mla_out_proj(
+        ctypes.byref(dims), _ptr(o, torch.bfloat16, "o"), _ptr(w_o, torch.bfloat16, "w_o"),
+        _ptr(y, torch.bfloat16, "y"), T, _stream(stream))
+    _check(st, "mla_out_proj")
 
 
 def mla_status_read(dev_status, stream=None) -> int:

@@ -9,6 +9,7 @@
 namespace {
 
 constexpr float kDefaultTheta = 10000.f;
+constexpr int32_t kMaxOutProjTokens = 1 << 20;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -160,6 +161,21 @@ int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16*
     if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
   }
   return cuda_status(mla::launch_decode_combine(a, s));
+}
+
+int mla_out_proj(const mla_dims* dims, const mla_bf16* o, const mla_bf16* w_o, mla_bf16* y,
+                 int32_t n_tokens, void* stream) {
+  int st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (n_tokens < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > kMaxOutProjTokens) return MLA_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return MLA_OK;
+  if (!o || !w_o || !y) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(y)) return MLA_ERR_MISALIGNED;
+  mla::OutProjArgs a;
+  a.x = o; a.w_o = w_o; a.y = y;
+  a.T = n_tokens; a.K = dims->n_heads * dims->v_head; a.D = dims->d_model;
+  return cuda_status(mla::launch_out_proj(a, (cudaStream_t)stream));
 }
 
 int mla_status_read(const int32_t* dev_status, void* stream) {

@@ -51,6 +51,13 @@ struct AbsorbArgs {
   double inv_freq[kMaxRopePairs];
 };
 
+struct OutProjArgs {
+  const uint16_t* x;          // [T, K] the heads' outputs, head-major (K = H * d_v)
+  const uint16_t* w_o;        // [D, K]
+  uint16_t* y;                // [T, D]
+  int T, K, D;
+};
+
 size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);
 int decode_simt_row_groups(int rows_total);
 cudaError_t launch_decode_split_simt(const DecodeArgs& a, cudaStream_t stream);
@@ -73,5 +80,6 @@ inline cudaLaunchAttribute pdl_attribute() {
 }
 cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
+cudaError_t launch_out_proj(const OutProjArgs& a, cudaStream_t stream);
 
 }  // namespace mla

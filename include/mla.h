@@ -197,6 +197,29 @@ int mla_decode_attn_noalloc(const mla_dims* dims, const mla_bf16* q_lat, const m
                             int32_t nq, int32_t max_pages, int32_t num_pages, const mla_bf16* w_uv,
                             mla_bf16* out, float* lse, int32_t* dev_status, void* stream);
 
+/*
+ * mla_out_proj - layer output projection of the step's tokens.
+ *
+ * For each token t and output feature i (0 <= i < d_model):
+ *   y[t][i] = sum_{h < H, j < v_head} w_o[i][h * v_head + j] * o[t][h][j]
+ * i.e. y = W_O concat_h(o_h), the heads' outputs concatenated head after head
+ * ([distaisys] sec. 3, out_proj of width H * d_h -> d_model, no bias).  Because
+ * mla_decode_attn applies W_UV once after attending over the latents, W_UV and
+ * W_O act back to back here ([from-scratch] "Absorption, and why RoPE breaks it":
+ * they fold into one matrix by associativity); this call keeps them separate so
+ * that `o` stays available per head.
+ *
+ *   o     device bf16 [n_tokens, H, v_head]; the `out` of mla_decode_attn
+ *         ([batch, nq, H, v_head]) with n_tokens = batch * nq
+ *   w_o   device bf16 [d_model, H * v_head]
+ *   y     device bf16 [n_tokens, d_model] (output; must not overlap o or w_o)
+ * fp32 accumulation, one bf16 rounding per output.  n_tokens == 0 is a no-op;
+ * n_tokens > 2^20 returns MLA_ERR_UNSUPPORTED.  The weight is streamed once per
+ * 32 tokens (once per call for n_tokens <= 32).
+ */
+int mla_out_proj(const mla_dims* dims, const mla_bf16* o, const mla_bf16* w_o, mla_bf16* y,
+                 int32_t n_tokens, void* stream);
+
 /* mla_status_read - wait for `stream`, then return the mla_status recorded in the
  * device word dev_status (MLA_OK if none), or MLA_ERR_CUDA if the copy failed. */
 int mla_status_read(const int32_t* dev_status, void* stream);

@@ -121,3 +121,18 @@ def test_workspace_query_rejects_bad_arguments(lib):
 def test_status_calls_reject_null(lib):
     assert lib.mla_status_read(None, None) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_status_clear(None, None) == M.MLA_ERR_INVALID_ARG
+
+
+def test_out_proj_argument_checks(lib):
+    d = v3_dims()
+    call = lambda **kw: lib.mla_out_proj(
+        ctypes.byref(d) if kw.get("dims", True) else None, kw.get("o", FAKE), kw.get("w", FAKE),
+        kw.get("y", FAKE), kw.get("T", 16), None)
+    assert call(dims=False) == M.MLA_ERR_INVALID_ARG
+    assert call(o=None) == M.MLA_ERR_INVALID_ARG
+    assert call(w=None) == M.MLA_ERR_INVALID_ARG
+    assert call(y=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(w=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(T=-1) == M.MLA_ERR_INVALID_ARG
+    assert call(T=(1 << 20) + 1) == M.MLA_ERR_UNSUPPORTED
+    assert call(T=0, o=None, y=None) == M.MLA_OK                      # empty: no-op

@@ -27,6 +27,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "DecodeInputs", "bf16_bits", "bf16_to_f32",
     "rng_for", "context_lengths", "make_page_table", "make_decode_inputs",
+    "make_out_proj_inputs",
 ]
 
 
@@ -104,8 +105,9 @@ def _normal(seed: int, name: str, shape, std: float = 1.0) -> np.ndarray:
     return out
 
 
-def _normal_bf16(seed: int, name: str, shape, chunk: int = 1 << 22) -> np.ndarray:
-    """N(0,1) draws rounded to bf16 for the large latent-cache pools.
+def _normal_bf16(seed: int, name: str, shape, chunk: int = 1 << 22, std: float = 1.0) -> np.ndarray:
+    """N(0, std^2) draws rounded to bf16 for the large tensors (latent-cache
+    pools, the output projection).
 
     The tensor is cut into chunks of `chunk` elements; chunk k draws from its own
     PCG64 stream keyed by (seed, name, k), so the values do not depend on how many
@@ -120,7 +122,10 @@ def _normal_bf16(seed: int, name: str, shape, chunk: int = 1 << 22) -> np.ndarra
         s = k * chunk
         n = min(chunk, out.size - s)
         g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, key, k])))
-        out[s:s + n] = bf16_bits(g.standard_normal(size=n, dtype=np.float32))
+        v = g.standard_normal(size=n, dtype=np.float32)
+        if std != 1.0:
+            v *= np.float32(std)
+        out[s:s + n] = bf16_bits(v)
 
     nchunks = (out.size + chunk - 1) // chunk
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
@@ -234,3 +239,17 @@ def make_decode_inputs(w: Workload, seed: int = 0, spare_pages: int = 0,
     if not w.fp32_values:
         raw = {}
     return DecodeInputs(w, seed, lens, seq_idx, pos, h_seq_idx, h_pos, table, num_pages, bits, raw)
+
+
+def make_out_proj_inputs(w: Workload, seed: int = 0, n_tokens: int | None = None) -> dict:
+    """Inputs of the layer output projection y = W_O concat_h(o_h) (bf16 bits):
+      o    [T, H, v_head]       the heads' attention outputs, N(0, 1)
+      w_o  [D, H * v_head]      out_proj weight, N(0, 1/fan_in) with fan_in = H * v_head
+                                (in_features of out_proj, distaisys.com deep-dive sec. 3)
+    T defaults to the workload's query tokens (batch * nq)."""
+    T = w.tokens if n_tokens is None else int(n_tokens)
+    K = w.n_heads * w.v_head
+    return {
+        "o": bf16_bits(_normal(seed, "attn_out", (T, w.n_heads, w.v_head))),
+        "w_o": _normal_bf16(seed, "w_o", (w.d_model, K), std=1.0 / np.sqrt(K)),
+    }
