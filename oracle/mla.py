@@ -245,6 +245,43 @@ def attend_brute(q, q_pos, C, KR, w_uk, w_uv, scale, theta=DEFAULT_THETA):
 
 
 # ----------------------------------------------------------------------------
+# Query path with low-rank query compression (q-LoRA)
+# ----------------------------------------------------------------------------
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value (8 significant bits,
+    ties to even), returned as float64.  One rounding straight from float64.
+    Normal range only (|x| >= 2^-126 or 0); inf and nan pass through."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                              # x = m 2^e, 0.5 <= |m| < 1
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)    # np.rint: half to even
+    return np.where(np.isfinite(x), r, x)
+
+
+def query_project(h: np.ndarray, w_dq: np.ndarray, w_uq: np.ndarray, n_heads: int,
+                  latent_bf16: bool = True):
+    """Queries from the hidden state through the compressed query latent.
+
+    c_Q = W_DQ h (width q_lora_rank, 1536 in the V3-shaped configuration of
+    [eyestech-blog] sec. 3), then [q_nope || q_rope] = W_UQ c_Q for every head
+    ([songhuiming] "Note on Actual Implementation": the query side is also
+    down-projected, then up-projected).  The pages name no normalisation
+    between the two maps; none is applied.  With latent_bf16, c_Q is rounded to
+    bf16 before the up-projection, as in the bf16 module of [eyestech-blog] sec. 3.
+
+    h [T, D]; w_dq [d_cq, D]; w_uq [H * (d_h + d_rope), d_cq] (rows head-major,
+    per head the non-rotary rows first).  Returns (c_q [T, d_cq],
+    q [T, H, d_h + d_rope]); q's RoPE part is not rotated yet.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    c_q = h @ np.asarray(w_dq, dtype=np.float64).T
+    if latent_bf16:
+        c_q = round_bf16(c_q)
+    q = c_q @ np.asarray(w_uq, dtype=np.float64).T
+    return c_q, q.reshape(h.shape[0], n_heads, q.shape[1] // n_heads)
+
+
+# ----------------------------------------------------------------------------
 # Layer output projection
 # ----------------------------------------------------------------------------
 
