@@ -20,9 +20,12 @@ positions, lengths) copied from pinned host memory and its output copied back,
 inside the timed region, double-buffered on a second stream the way a serving
 loop overlaps transfers with the neighbouring steps' compute.
 
-next_rows.out_proj: the layer output projection y = W_O concat_h(o_h)
-(mla_out_proj) on the step's output, timed alone after the step (it is not part
-of the step); W_O (235 MB at the V3 shape) is larger than L2.
+next_rows: the layer output projection y = W_O concat_h(o_h) (mla_out_proj, on
+the step's output) and the q-LoRA query path c_Q = W_DQ h, q = W_UQ c_Q
+(mla_query_proj, q_lora_rank 1536), each timed alone after the step (neither is
+part of the step); W_O (235 MB at the V3 shape) is larger than L2, W_DQ + W_UQ
+(97.5 MB) are not, so an L2-sized buffer is rewritten before each timed call of
+the query path.
 
 --impl reference times the CPU oracle (float64 numpy, absorbed form) on a
 bounded sample of the same workload on the host cores, as the comparison arm.
@@ -310,13 +313,45 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
     assert torch.equal(out_host[(args.steps - 1) % 2], outs[(args.steps - 1) % 2].cpu()), "e2e output copy"
 
     op = measure_out_proj(M, w, dims, out, dev, stream, args.seed + rank)
+    qp = measure_query_proj(M, w, dims, dev, stream, args.seed + rank)
 
-    ms_total, e2e_ms, dec_ms, op_us = max_over_ranks(
-        [ms_total, e2e_ms, float(np.mean(decode_ms)), op["time_us"]], dev)
+    ms_total, e2e_ms, dec_ms, op_us, qp_us = max_over_ranks(
+        [ms_total, e2e_ms, float(np.mean(decode_ms)), op["time_us"], qp["time_us"]], dev)
     op["time_us"] = op_us
+    qp["time_us"] = qp_us
     return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": dec_ms, "clocks": clocks,
             "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens,
-            "out_proj": op}
+            "out_proj": op, "query_proj": qp}
+
+
+def measure_query_proj(M, w: W.Workload, dims, dev, stream, seed: int, iters: int = 50) -> dict:
+    """Average device time of mla_query_proj (its two launches) with a 256 MB
+    buffer rewritten between calls, so that the weights come from HBM each time;
+    each call is bracketed by its own CUDA events on the launching stream."""
+    import torch
+    r = W.Q_LORA_RANK
+    x = W.make_query_proj_inputs(w, seed, w.tokens, r)
+    h, w_dq, w_uq = (torch.from_numpy(x[k]).view(torch.bfloat16).to(dev) for k in ("h", "w_dq", "w_uq"))
+    c_q = torch.empty((w.tokens, r), dtype=torch.bfloat16, device=dev)
+    q = torch.empty((w.tokens, w.n_heads, w.qk_nope + w.d_rope), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        M.mla_query_proj(dims, h, w_dq, w_uq, c_q, q, stream=stream)
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(iters):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        M.mla_query_proj(dims, h, w_dq, w_uq, c_q, q, stream=stream)
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    us = float(np.mean([a.elapsed_time(b) for a, b in times])) * 1000.0
+    nbytes = (w_dq.numel() + w_uq.numel() + h.numel() + 2 * c_q.numel() + q.numel()) * 2
+    return {"time_us": us, "bytes_per_launch": nbytes, "launches": 2 * iters, "tokens": w.tokens,
+            "shape": f"c_Q[{w.tokens}, {r}] = h[{w.tokens}, {w.d_model}] . W_DQ^T; "
+                     f"q[{w.tokens}, {w.n_heads}, {w.qk_nope + w.d_rope}] = c_Q . W_UQ^T"}
 
 
 def measure_out_proj(M, w: W.Workload, dims, out, dev, stream, seed: int, iters: int = 50) -> dict:
@@ -480,10 +515,17 @@ def main():
     op = r["out_proj"]
     op_gbs = op["bytes_per_launch"] / (op["time_us"] * 1e-6) / 1e9
     line["next_rows"] = {"out_proj": {
-        "kernel": "out_proj_kernel (mla_out_proj), timed alone after the step, not part of it",
+        "kernel": "token_linear_kernel (mla_out_proj), timed alone after the step, not part of it",
         "shape": op["shape"], "bound": "hbm", "achieved": op_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": op_gbs / peaks["hbm_gbs"], "time_us": op["time_us"], "bytes_per_launch": op["bytes_per_launch"],
         "launches_timed": op["launches"], "l2": "W_O is larger than L2"}}
+    qp = r["query_proj"]
+    qp_gbs = qp["bytes_per_launch"] / (qp["time_us"] * 1e-6) / 1e9
+    line["next_rows"]["query_proj"] = {
+        "kernel": "token_linear_kernel x 2 (mla_query_proj), timed alone after the step, not part of it",
+        "shape": qp["shape"], "bound": "hbm", "achieved": qp_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": qp_gbs / peaks["hbm_gbs"], "time_us": qp["time_us"], "bytes_per_call": qp["bytes_per_launch"],
+        "launches_timed": qp["launches"], "l2": "256 MB buffer rewritten before each call"}
     if world == 1 and not args.no_cpu_baseline:
         arm = OracleArm(w, args.seed)
         v, sample = arm.measure(args.cpu_budget)

@@ -40,6 +40,7 @@ SIGNATURES = {
                                        _P, _P, _P, _P]),
     "mla_decode_attn_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "mla_out_proj": (ctypes.c_int, [_P, _P, _P, _P, _I, _P]),
+    "mla_query_proj": (ctypes.c_int, [_P, _I, _P, _P, _P, _P, _P, _I, _P]),
     "mla_status_read": (ctypes.c_int, [_P, _P]),
     "mla_status_clear": (ctypes.c_int, [_P, _P]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -251,6 +252,23 @@ def mla_out_proj(dims: MlaDims, o, w_o, y, stream=None) -> None:
         ctypes.byref(dims), _ptr(o, torch.bfloat16, "o"), _ptr(w_o, torch.bfloat16, "w_o"),
         _ptr(y, torch.bfloat16, "y"), T, _stream(stream))
     _check(st, "mla_out_proj")
+
+
+def mla_query_proj(dims: MlaDims, h, w_dq, w_uq, c_q, q, stream=None) -> None:
+    """c_q [T, q_lora_rank] = W_DQ h, then q [T, H, qk_nope + d_rope] = W_UQ c_q."""
+    torch = _torch()
+    T = h.shape[0]
+    r = w_dq.shape[0]
+    _shape(h, (T, dims.d_model), "h")
+    _shape(w_dq, (r, dims.d_model), "w_dq")
+    _shape(w_uq, (dims.n_heads * (dims.qk_nope + dims.d_rope), r), "w_uq")
+    _shape(c_q, (T, r), "c_q")
+    _shape(q, (T, dims.n_heads, dims.qk_nope + dims.d_rope), "q")
+    st = load_library().mla_query_proj(
+        ctypes.byref(dims), r, _ptr(h, torch.bfloat16, "h"), _ptr(w_dq, torch.bfloat16, "w_dq"),
+        _ptr(w_uq, torch.bfloat16, "w_uq"), _ptr(c_q, torch.bfloat16, "c_q"), _ptr(q, torch.bfloat16, "q"),
+        T, _stream(stream))
+    _check(st, "mla_query_proj")
 
 
 def mla_status_read(dev_status, stream=None) -> int:

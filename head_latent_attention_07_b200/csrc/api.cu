@@ -9,7 +9,8 @@
 namespace {
 
 constexpr float kDefaultTheta = 10000.f;
-constexpr int32_t kMaxOutProjTokens = 1 << 20;
+constexpr int32_t kMaxOutProjTokens = 1 << 20;   // tokens of one out / query projection call
+constexpr int32_t kMaxQLoraRank = 1 << 16;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -172,10 +173,38 @@ int mla_out_proj(const mla_dims* dims, const mla_bf16* o, const mla_bf16* w_o, m
   if (n_tokens == 0) return MLA_OK;
   if (!o || !w_o || !y) return MLA_ERR_INVALID_ARG;
   if (!aligned16(o) || !aligned16(w_o) || !aligned16(y)) return MLA_ERR_MISALIGNED;
-  mla::OutProjArgs a;
-  a.x = o; a.w_o = w_o; a.y = y;
-  a.T = n_tokens; a.K = dims->n_heads * dims->v_head; a.D = dims->d_model;
-  return cuda_status(mla::launch_out_proj(a, (cudaStream_t)stream));
+  int sms = 0;
+  if ((st = device_sms(&sms)) != MLA_OK) return st;
+  mla::LinearArgs a;
+  a.x = o; a.w = w_o; a.y = y;
+  a.T = n_tokens; a.K = dims->n_heads * dims->v_head; a.N = dims->d_model;
+  a.ksplit = mla::linear_ksplit(a.N, a.K, sms);
+  return cuda_status(mla::launch_linear(a, (cudaStream_t)stream));
+}
+
+int mla_query_proj(const mla_dims* dims, int32_t q_lora_rank, const mla_bf16* h, const mla_bf16* w_dq,
+                   const mla_bf16* w_uq, mla_bf16* c_q, mla_bf16* q, int32_t n_tokens, void* stream) {
+  int st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (n_tokens < 0 || q_lora_rank < 1) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > kMaxOutProjTokens || q_lora_rank % 8 || q_lora_rank > kMaxQLoraRank) return MLA_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return MLA_OK;
+  if (!h || !w_dq || !w_uq || !c_q || !q) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_dq) || !aligned16(w_uq) || !aligned16(c_q) || !aligned16(q))
+    return MLA_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_sms(&sms)) != MLA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  mla::LinearArgs down;                        // c_Q = W_DQ h
+  down.x = h; down.w = w_dq; down.y = c_q;
+  down.T = n_tokens; down.K = dims->d_model; down.N = q_lora_rank;
+  down.ksplit = mla::linear_ksplit(down.N, down.K, sms);
+  if ((st = cuda_status(mla::launch_linear(down, s))) != MLA_OK) return st;
+  mla::LinearArgs up;                          // [q_nope || q_rope] per head = W_UQ c_Q
+  up.x = c_q; up.w = w_uq; up.y = q;
+  up.T = n_tokens; up.K = q_lora_rank; up.N = dims->n_heads * (dims->qk_nope + dims->d_rope);
+  up.ksplit = mla::linear_ksplit(up.N, up.K, sms);
+  return cuda_status(mla::launch_linear(up, s));
 }
 
 int mla_status_read(const int32_t* dev_status, void* stream) {

@@ -28,6 +28,9 @@ __global__ void __launch_bounds__(kAppWarps * 32)
 append_latent_kernel(AppendArgs a) {
   __shared__ float part[kAppWarps][16][17];
   __shared__ float red[kAppSplit][16][17];   // cluster leader: the split CTAs' tiles
+  // split cluster barrier: the wait before the first remote store below makes sure
+  // every CTA of the cluster (the leader included) has started
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   allow_dependent_launch();
   grid_dependency_wait();
   const int R = a.d_c + a.d_rope;
@@ -69,6 +72,7 @@ append_latent_kernel(AppendArgs a) {
     part[warp][row][tok + 8] = d1[e];
   }
   __syncthreads();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   {
     // this CTA's tile -> slot `split` of the leader's shared memory
     const int row = threadIdx.x >> 4, tok = threadIdx.x & 15;

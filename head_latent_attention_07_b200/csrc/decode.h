@@ -51,11 +51,13 @@ struct AbsorbArgs {
   double inv_freq[kMaxRopePairs];
 };
 
-struct OutProjArgs {
-  const uint16_t* x;          // [T, K] the heads' outputs, head-major (K = H * d_v)
-  const uint16_t* w_o;        // [D, K]
-  uint16_t* y;                // [T, D]
-  int T, K, D;
+// y[T, N] = x[T, K] W[N, K]^T for a few tokens (the query projections, W_O)
+struct LinearArgs {
+  const uint16_t* x;          // [T, K]
+  const uint16_t* w;          // [N, K]
+  uint16_t* y;                // [T, N]
+  int T, K, N;
+  int ksplit;                 // CTAs of a cluster splitting K (1, 2, 4 or 8)
 };
 
 size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);
@@ -80,6 +82,7 @@ inline cudaLaunchAttribute pdl_attribute() {
 }
 cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
-cudaError_t launch_out_proj(const OutProjArgs& a, cudaStream_t stream);
+int linear_ksplit(int N, int K, int sms);
+cudaError_t launch_linear(const LinearArgs& a, cudaStream_t stream);
 
 }  // namespace mla

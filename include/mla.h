@@ -7,6 +7,9 @@
  *   mla_absorb_q       fold W_UK into the queries, rotate their RoPE part
  *   mla_decode_attn    split-KV attention over the paged latent cache,
  *                      log-sum-exp combine of the splits, then W_UV
+ * Around them: mla_query_proj (the queries from the hidden state through the
+ * compressed query latent, before mla_absorb_q) and mla_out_proj (the layer
+ * output W_O concat_h(o_h), after mla_decode_attn).
  * Keys and values are never decompressed: every cached token holds only its
  * latent c_t (d_c scalars) and its decoupled RoPE key k_t^R (d_rope scalars).
  *
@@ -219,6 +222,30 @@ int mla_decode_attn_noalloc(const mla_dims* dims, const mla_bf16* q_lat, const m
  */
 int mla_out_proj(const mla_dims* dims, const mla_bf16* o, const mla_bf16* w_o, mla_bf16* y,
                  int32_t n_tokens, void* stream);
+
+/*
+ * mla_query_proj - queries through the compressed query latent (q-LoRA).
+ *
+ * For each token t:
+ *   c_q[t] = bf16(W_DQ h[t])               width q_lora_rank (1536 in the V3-shaped
+ *                                          decoder of [eyestech-blog] sec. 3)
+ *   q[t]   = bf16(W_UQ c_q[t]) as [H][qk_nope + d_rope], per head q_nope then q_rope
+ * ([songhuiming] "Note on Actual Implementation": the query side is down- then
+ * up-projected).  The pages name no normalisation between the two maps; none is
+ * applied.  c_q is rounded to bf16 before the up-projection (a bf16 module's
+ * activation) and is returned.  q is the input of mla_absorb_q (RoPE not applied).
+ *
+ *   h     device bf16 [n_tokens, d_model]
+ *   w_dq  device bf16 [q_lora_rank, d_model]
+ *   w_uq  device bf16 [H * (qk_nope + d_rope), q_lora_rank]; rows head-major
+ *   c_q   device bf16 [n_tokens, q_lora_rank] (output)
+ *   q     device bf16 [n_tokens, H, qk_nope + d_rope] (output)
+ * fp32 accumulation.  q_lora_rank must be a multiple of 8 (<= 65536); n_tokens ==
+ * 0 is a no-op; n_tokens > 2^20 returns MLA_ERR_UNSUPPORTED.  Outputs must not
+ * overlap the inputs.  Two kernels, in order, on `stream`.
+ */
+int mla_query_proj(const mla_dims* dims, int32_t q_lora_rank, const mla_bf16* h, const mla_bf16* w_dq,
+                   const mla_bf16* w_uq, mla_bf16* c_q, mla_bf16* q, int32_t n_tokens, void* stream);
 
 /* mla_status_read - wait for `stream`, then return the mla_status recorded in the
  * device word dev_status (MLA_OK if none), or MLA_ERR_CUDA if the copy failed. */

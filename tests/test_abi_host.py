@@ -136,3 +136,18 @@ def test_out_proj_argument_checks(lib):
     assert call(T=-1) == M.MLA_ERR_INVALID_ARG
     assert call(T=(1 << 20) + 1) == M.MLA_ERR_UNSUPPORTED
     assert call(T=0, o=None, y=None) == M.MLA_OK                      # empty: no-op
+
+
+def test_query_proj_argument_checks(lib):
+    d = v3_dims()
+    call = lambda **kw: lib.mla_query_proj(
+        ctypes.byref(d), kw.get("r", 1536), kw.get("h", FAKE), kw.get("wdq", FAKE), kw.get("wuq", FAKE),
+        kw.get("c", FAKE), kw.get("q", FAKE), kw.get("T", 16), None)
+    assert call(h=None) == M.MLA_ERR_INVALID_ARG
+    assert call(q=None) == M.MLA_ERR_INVALID_ARG
+    assert call(r=0) == M.MLA_ERR_INVALID_ARG
+    assert call(r=1540) == M.MLA_ERR_UNSUPPORTED                    # rows of w_uq must stay 16-byte aligned
+    assert call(c=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(wuq=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(T=-1) == M.MLA_ERR_INVALID_ARG
+    assert call(T=0, h=None, q=None) == M.MLA_OK                     # empty: no-op

@@ -27,7 +27,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "DecodeInputs", "bf16_bits", "bf16_to_f32",
     "rng_for", "context_lengths", "make_page_table", "make_decode_inputs",
-    "make_out_proj_inputs",
+    "make_out_proj_inputs", "make_query_proj_inputs", "Q_LORA_RANK",
 ]
 
 
@@ -239,6 +239,26 @@ def make_decode_inputs(w: Workload, seed: int = 0, spare_pages: int = 0,
     if not w.fp32_values:
         raw = {}
     return DecodeInputs(w, seed, lens, seq_idx, pos, h_seq_idx, h_pos, table, num_pages, bits, raw)
+
+
+# q_lora_rank of the V3-shaped decoder (eyestech.in MLA article, sec. 3)
+Q_LORA_RANK = 1536
+
+
+def make_query_proj_inputs(w: Workload, seed: int = 0, n_tokens: int | None = None,
+                           q_lora_rank: int = Q_LORA_RANK) -> dict:
+    """Inputs of the q-LoRA query path c_Q = W_DQ h, q = W_UQ c_Q (bf16 bits):
+      h     [T, D]                          hidden states, N(0, 1)
+      w_dq  [q_lora_rank, D]                N(0, 1/D)
+      w_uq  [H * (qk_nope + d_rope), q_lora_rank]   N(0, 1/q_lora_rank)
+    (fan_in = in_features, as for the other projections).  T defaults to batch * nq."""
+    T = w.tokens if n_tokens is None else int(n_tokens)
+    n_q = w.n_heads * (w.qk_nope + w.d_rope)
+    return {
+        "h": bf16_bits(_normal(seed, "q_path_h", (T, w.d_model))),
+        "w_dq": _normal_bf16(seed, "w_dq", (q_lora_rank, w.d_model), std=1.0 / np.sqrt(w.d_model)),
+        "w_uq": _normal_bf16(seed, "w_uq", (n_q, q_lora_rank), std=1.0 / np.sqrt(q_lora_rank)),
+    }
 
 
 def make_out_proj_inputs(w: Workload, seed: int = 0, n_tokens: int | None = None) -> dict:
