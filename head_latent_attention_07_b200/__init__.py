@@ -39,6 +39,10 @@ SIGNATURES = {
     "mla_decode_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, ctypes.c_size_t,
                                        _P, _P, _P, _P]),
     "mla_decode_attn_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "mla_decode_attn_partial": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, ctypes.c_size_t,
+                                               _P, _P, _P, _P]),
+    "mla_merge_ranks": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p), _I, _I,
+                                       _P, _P, _P, _P]),
     "mla_out_proj": (ctypes.c_int, [_P, _P, _P, _P, _I, _P]),
     "mla_query_proj": (ctypes.c_int, [_P, _I, _P, _P, _P, _P, _P, _I, _P]),
     "mla_status_read": (ctypes.c_int, [_P, _P]),
@@ -237,6 +241,55 @@ def mla_decode_attn_noalloc(dims: MlaDims, q_lat, pool, page_table, seq_lens, w_
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
         _ptr(dev_status, torch.int32, "dev_status"), _stream(stream))
     _check(st, "mla_decode_attn_noalloc")
+
+
+def mla_decode_attn_partial(dims: MlaDims, q_lat, pool, page_table, seq_lens, kv_rank: int, kv_ranks: int,
+                            workspace, o_lat, lse, dev_status=None, stream=None) -> None:
+    """Rank kv_rank's window of a context-split decode: o_lat [B, nq, H, d_c] (fp32)
+    and lse [B, nq, H] over pages [P_b r / R, P_b (r+1) / R) of each sequence."""
+    torch = _torch()
+    B, nq = q_lat.shape[0], q_lat.shape[1]
+    _shape(q_lat, (B, nq, dims.n_heads, dims.row), "q_lat")
+    num_pages = pool.shape[0]
+    _shape(pool, (num_pages, dims.page_size, dims.row), "pool")
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, max_pages]")
+    _shape(seq_lens, (B,), "seq_lens")
+    _shape(o_lat, (B, nq, dims.n_heads, dims.d_c), "o_lat")
+    _shape(lse, (B, nq, dims.n_heads), "lse")
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1:
+        raise TypeError("workspace must be a 1-D uint8 tensor")
+    st = load_library().mla_decode_attn_partial(
+        ctypes.byref(dims), _ptr(q_lat, torch.bfloat16, "q_lat"), _ptr(pool, torch.bfloat16, "pool"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        B, nq, page_table.shape[1], num_pages, kv_rank, kv_ranks,
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _ptr(o_lat, torch.float32, "o_lat"), _ptr(lse, torch.float32, "lse"),
+        _ptr(dev_status, torch.int32, "dev_status"), _stream(stream))
+    _check(st, "mla_decode_attn_partial")
+
+
+def mla_merge_ranks(dims: MlaDims, o_lats, lses, w_uv, out, lse=None, stream=None) -> None:
+    """Merge the ranks' (o_lat [T, H, d_c], lse [T, H]) partials by log-sum-exp, then
+    W_UV: out [T, H, v_head].  o_lats / lses are sequences of tensors (one per rank;
+    [B, nq, ...] shapes are accepted as T = B * nq)."""
+    torch = _torch()
+    R = len(o_lats)
+    if R != len(lses) or R < 1:
+        raise ValueError("one o_lat and one lse per rank")
+    T = out.numel() // (dims.n_heads * dims.v_head)
+    _shape(out.view(T, dims.n_heads, dims.v_head), (T, dims.n_heads, dims.v_head), "out")
+    for o, l in zip(o_lats, lses):
+        if o.numel() != T * dims.n_heads * dims.d_c or l.numel() != T * dims.n_heads:
+            raise ValueError("partials must be [T, H, d_c] and [T, H]")
+    if lse is not None and lse.numel() != T * dims.n_heads:
+        raise ValueError("lse must hold T * H values")
+    po = (ctypes.c_void_p * R)(*[_ptr(o, torch.float32, "o_lat").value for o in o_lats])
+    pl = (ctypes.c_void_p * R)(*[_ptr(l, torch.float32, "lse").value for l in lses])
+    st = load_library().mla_merge_ranks(
+        ctypes.byref(dims), po, pl, R, T, _ptr(w_uv, torch.bfloat16, "w_uv"), _ptr(out, torch.bfloat16, "out"),
+        _ptr(lse, torch.float32, "lse"), _stream(stream))
+    _check(st, "mla_merge_ranks")
 
 
 def mla_out_proj(dims: MlaDims, o, w_o, y, stream=None) -> None:

@@ -11,6 +11,7 @@ namespace {
 constexpr float kDefaultTheta = 10000.f;
 constexpr int32_t kMaxOutProjTokens = 1 << 20;   // tokens of one out / query projection call
 constexpr int32_t kMaxQLoraRank = 1 << 16;
+constexpr int32_t kMaxMergeTokens = 1 << 18;     // grid rows of the rank merge stay below 65536
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -122,20 +123,27 @@ size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n
   return ws_layout(dims, batch, nq, sms).total;
 }
 
-int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
-                    const int32_t* page_table, const int32_t* seq_lens, int32_t batch,
-                    int32_t nq, int32_t max_pages, int32_t num_pages, const mla_bf16* w_uv,
-                    void* workspace, size_t ws_bytes, mla_bf16* out, float* lse,
-                    int32_t* dev_status, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The decode path of mla_decode_attn (out set) and mla_decode_attn_partial
+// (o_lat set: the combine writes the merged latent output of this rank's window).
+int decode_common(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool, const int32_t* page_table,
+                  const int32_t* seq_lens, int32_t batch, int32_t nq, int32_t max_pages, int32_t num_pages,
+                  const mla_bf16* w_uv, int32_t kv_rank, int32_t kv_ranks, void* workspace, size_t ws_bytes,
+                  mla_bf16* out, float* o_lat, float* lse, int32_t* dev_status, void* stream) {
   int st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (batch < 1 || nq < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (kv_ranks < 1 || kv_rank < 0 || kv_rank >= kv_ranks) return MLA_ERR_INVALID_ARG;
   if (batch > mla::kMaxBatch || nq > 16) return MLA_ERR_UNSUPPORTED;
   if ((int64_t)max_pages * dims->page_size > INT32_MAX) return MLA_ERR_UNSUPPORTED;
-  if (!q_lat || !pool || !page_table || !seq_lens || !w_uv || !workspace || !out) return MLA_ERR_INVALID_ARG;
+  if (!q_lat || !pool || !page_table || !seq_lens || !workspace || (!out && !o_lat)) return MLA_ERR_INVALID_ARG;
+  if (out && !w_uv) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_lat) || !aligned16(pool) || !aligned16(page_table) || !aligned16(seq_lens) ||
-      !aligned16(w_uv) || !aligned16(workspace) || !aligned16(out) || (lse && !aligned16(lse)) ||
-      (dev_status && !aligned16(dev_status)))
+      (w_uv && !aligned16(w_uv)) || !aligned16(workspace) || (out && !aligned16(out)) ||
+      (o_lat && !aligned16(o_lat)) || (lse && !aligned16(lse)) || (dev_status && !aligned16(dev_status)))
     return MLA_ERR_MISALIGNED;
   int sms = 0;
   if ((st = device_sms(&sms)) != MLA_OK) return st;
@@ -144,12 +152,13 @@ int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16*
 
   mla::DecodeArgs a;
   a.q_lat = q_lat; a.pool = pool; a.page_table = page_table; a.seq_lens = seq_lens; a.w_uv = w_uv;
-  a.out = out; a.lse = lse; a.dev_status = dev_status;
+  a.out = out; a.lse = lse; a.dev_status = dev_status; a.out_lat = o_lat;
   a.part_o = reinterpret_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + wl.part_o_bytes);
   a.batch = batch; a.nq = nq; a.n_heads = dims->n_heads; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
   a.v_head = dims->v_head; a.page_size = dims->page_size; a.max_pages = max_pages;
   a.num_pages = num_pages; a.scale = eff_scale(dims);
+  a.kv_rank = kv_rank; a.kv_ranks = kv_ranks;
   cudaStream_t s = (cudaStream_t)stream;
   if (mla::decode_tc_supported(dims->d_c, dims->d_rope, dims->page_size)) {
     // tensor-core path: one CTA pair per worker and 128-row tile
@@ -162,6 +171,54 @@ int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16*
     if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
   }
   return cuda_status(mla::launch_decode_combine(a, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
+                    const int32_t* page_table, const int32_t* seq_lens, int32_t batch,
+                    int32_t nq, int32_t max_pages, int32_t num_pages, const mla_bf16* w_uv,
+                    void* workspace, size_t ws_bytes, mla_bf16* out, float* lse,
+                    int32_t* dev_status, void* stream) {
+  if (!out) return MLA_ERR_INVALID_ARG;
+  return decode_common(dims, q_lat, pool, page_table, seq_lens, batch, nq, max_pages, num_pages, w_uv, 0, 1,
+                       workspace, ws_bytes, out, nullptr, lse, dev_status, stream);
+}
+
+int mla_decode_attn_partial(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
+                            const int32_t* page_table, const int32_t* seq_lens, int32_t batch, int32_t nq,
+                            int32_t max_pages, int32_t num_pages, int32_t kv_rank, int32_t kv_ranks,
+                            void* workspace, size_t ws_bytes, float* o_lat, float* lse, int32_t* dev_status,
+                            void* stream) {
+  if (!o_lat || !lse) return MLA_ERR_INVALID_ARG;
+  return decode_common(dims, q_lat, pool, page_table, seq_lens, batch, nq, max_pages, num_pages, nullptr, kv_rank,
+                       kv_ranks, workspace, ws_bytes, nullptr, o_lat, lse, dev_status, stream);
+}
+
+int mla_merge_ranks(const mla_dims* dims, const float* const* o_lat, const float* const* lse, int32_t n_ranks,
+                    int32_t n_tokens, const mla_bf16* w_uv, mla_bf16* out, float* lse_out, void* stream) {
+  int st = check_dims(dims);
+  if (st != MLA_OK) return st;
+  if (n_tokens < 0 || n_ranks < 1 || !o_lat || !lse) return MLA_ERR_INVALID_ARG;
+  if (n_ranks > mla::kMaxRanks || n_tokens > kMaxMergeTokens) return MLA_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return MLA_OK;
+  if (!w_uv || !out) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(w_uv) || !aligned16(out) || (lse_out && !aligned16(lse_out))) return MLA_ERR_MISALIGNED;
+  mla::RankSources src = {};
+  src.n = n_ranks;
+  for (int r = 0; r < n_ranks; ++r) {
+    if (!o_lat[r] || !lse[r]) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(o_lat[r]) || !aligned16(lse[r])) return MLA_ERR_MISALIGNED;
+    src.o[r] = o_lat[r];
+    src.lse[r] = lse[r];
+  }
+  mla::DecodeArgs a = {};
+  a.w_uv = w_uv; a.out = out; a.lse = lse_out;
+  a.batch = n_tokens; a.nq = 1; a.n_heads = dims->n_heads; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
+  a.v_head = dims->v_head; a.page_size = dims->page_size; a.kv_ranks = 1;
+  return cuda_status(mla::launch_merge_ranks(a, src, (cudaStream_t)stream));
 }
 
 int mla_out_proj(const mla_dims* dims, const mla_bf16* o, const mla_bf16* w_o, mla_bf16* y,

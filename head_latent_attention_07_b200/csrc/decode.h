@@ -25,9 +25,22 @@ struct DecodeArgs {
   float* part_o;              // [pieces, nq*H, d_c]
   float* part_lse;            // [pieces, nq*H]
   int32_t* dev_status;        // or null
+  float* out_lat;             // [B, nq, H, d_c] or null: the combine writes the merged latent
+                              // output (and lse) instead of applying W_UV (context split)
   int batch, nq, n_heads, d_c, d_rope, v_head, page_size, max_pages, num_pages;
   int G;                      // split workers
+  int kv_rank, kv_ranks;      // context split: this call takes window kv_rank of kv_ranks
   float scale;
+};
+
+// Partials of the ranks of a context split, merged by launch_merge_ranks: rank
+// r's latent output [T, H, d_c] and lse [T, H] (device pointers: this GPU's
+// memory or a peer's).
+constexpr int kMaxRanks = 16;
+struct RankSources {
+  const float* o[kMaxRanks];
+  const float* lse[kMaxRanks];
+  int n;
 };
 
 struct AppendArgs {
@@ -64,6 +77,8 @@ size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);
 int decode_simt_row_groups(int rows_total);
 cudaError_t launch_decode_split_simt(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream);
+// LSE merge of the ranks' partials, then W_UV: a.batch = tokens, a.nq = 1.
+cudaError_t launch_merge_ranks(const DecodeArgs& a, const RankSources& src, cudaStream_t stream);
 
 // Tensor-core split kernel (d_c = 512, d_rope = 64, 64-token pages).
 bool decode_tc_supported(int d_c, int d_rope, int page_size);

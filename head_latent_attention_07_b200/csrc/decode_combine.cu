@@ -15,6 +15,12 @@
 // out.  At d_c = 512 and 16 query tokens this is 2 CTAs per head, all resident
 // at once (one wave at two CTAs per SM); the W_UV slice streams into shared
 // memory before the kernel waits for the split kernel's partials.
+//
+// Context split (one call per rank over a window of every sequence's pages):
+// with a.out_lat set, the kernel stops after the merge and writes the rank's
+// o_lat and lse; the rank-merge form (RANKS) then takes the ranks' partials as
+// its pieces (plain loads through the given pointers, which may point into a
+// peer GPU's memory) and finishes with W_UV as above.
 #include "common.cuh"
 #include "decode.h"
 #include "mma_frag.cuh"
@@ -51,8 +57,9 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t local_smem, uint32_t ra
   return v;
 }
 
+template <bool RANKS>
 __global__ void __launch_bounds__(kThreads, 2)
-decode_combine_kernel(DecodeArgs a, int KS) {
+decode_combine_kernel(DecodeArgs a, const __grid_constant__ RankSources src, int KS) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PlanSmem* ps = reinterpret_cast<PlanSmem*>(smem_raw);
   uint16_t* o_hi = reinterpret_cast<uint16_t*>(smem_raw + ((sizeof(PlanSmem) + 15) & ~size_t(15)));
@@ -86,14 +93,21 @@ decode_combine_kernel(DecodeArgs a, int KS) {
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
-  // The predecessor on the stream is always this call's split kernel, which
-  // writes only the partials and lets this kernel launch only after its own
-  // dependency wait: seq_lens and W_UV are final here, the partials after the
-  // wait below.
+  const bool lat_mode = !RANKS && a.out_lat != nullptr;
   allow_dependent_launch();
-  stage_w(0);
-  build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr);
-  grid_dependency_wait();   // the split kernel's partials
+  if (RANKS) {
+    // the predecessor is the caller's: wait before reading anything
+    grid_dependency_wait();
+    stage_w(0);
+  } else {
+    // The predecessor on the stream is always this call's split kernel, which
+    // writes only the partials and lets this kernel launch only after its own
+    // dependency wait: seq_lens and W_UV are final here, the partials after the
+    // wait below.
+    if (!lat_mode) stage_w(0);
+    build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr, a.kv_rank, a.kv_ranks);
+    grid_dependency_wait();   // the split kernel's partials
+  }
 
   // 1. merge: 16 threads per token, each owning columns [8 gc, 8 gc + 8) and
   //    [128 + 8 gc, 128 + 8 gc + 8) of the slice; one pass over the pieces in
@@ -108,8 +122,9 @@ decode_combine_kernel(DecodeArgs a, int KS) {
     if (t < T) {
       const int b = t / a.nq, i = t % a.nq;
       const int row = i * a.n_heads + h;
-      const int pb = ps->piece_begin[b];
-      const int np = ps->piece_begin[b + 1] - pb;
+      const size_t trow = (size_t)t * a.n_heads + h;   // row of a rank's partial [T, H, d_c]
+      const int pb = RANKS ? 0 : ps->piece_begin[b];
+      const int np = RANKS ? src.n : ps->piece_begin[b + 1] - pb;
       bool cols[2];
 #pragma unroll
       for (int half = 0; half < 2; ++half) cols[half] = 128 * half + 8 * gc < ncol;
@@ -124,14 +139,20 @@ decode_combine_kernel(DecodeArgs a, int KS) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) v[u][k] = make_float4(0.f, 0.f, 0.f, 0.f);
           if (s < np) {
-            const size_t pr = (size_t)(pb + s) * rows_total + row;
-            lv[u] = a.part_lse[pr];
-            const float* src = a.part_o + pr * a.d_c + col0 + 8 * gc;
+            const float* sp;
+            if (RANKS) {
+              lv[u] = src.lse[s][trow];
+              sp = src.o[s] + trow * a.d_c + col0 + 8 * gc;
+            } else {
+              const size_t pr = (size_t)(pb + s) * rows_total + row;
+              lv[u] = a.part_lse[pr];
+              sp = a.part_o + pr * a.d_c + col0 + 8 * gc;
+            }
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
               if (cols[half]) {
-                v[u][2 * half] = __ldcs(reinterpret_cast<const float4*>(src + 128 * half));
-                v[u][2 * half + 1] = __ldcs(reinterpret_cast<const float4*>(src + 128 * half + 4));
+                v[u][2 * half] = __ldcs(reinterpret_cast<const float4*>(sp + 128 * half));
+                v[u][2 * half + 1] = __ldcs(reinterpret_cast<const float4*>(sp + 128 * half + 4));
               }
             }
           }
@@ -162,8 +183,21 @@ decode_combine_kernel(DecodeArgs a, int KS) {
       const float inv = (m == -INFINITY) ? 0.f : 1.f / tot;
 #pragma unroll
       for (int e = 0; e < 16; ++e) acc[e] *= inv;
-      if (ks == 0 && gc == 0 && a.lse != nullptr) a.lse[(size_t)t * a.n_heads + h] = lse_all;
+      if (ks == 0 && gc == 0 && a.lse != nullptr) a.lse[trow] = lse_all;
+      if (lat_mode) {
+        // this rank's merged latent output, for the rank merge
+        float* dst = a.out_lat + trow * a.d_c + col0 + 8 * gc;
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+          if (cols[half]) {
+            *reinterpret_cast<float4*>(dst + 128 * half) =
+                make_float4(acc[8 * half], acc[8 * half + 1], acc[8 * half + 2], acc[8 * half + 3]);
+            *reinterpret_cast<float4*>(dst + 128 * half + 4) =
+                make_float4(acc[8 * half + 4], acc[8 * half + 5], acc[8 * half + 6], acc[8 * half + 7]);
+          }
+      }
     }
+    if (lat_mode) return;   // the whole grid takes this branch: no cluster barrier is left waiting
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       uint32_t hi[4], lo[4];
@@ -245,9 +279,13 @@ size_t decode_combine_smem_bytes(int d_c) {
          (size_t)kVChunk * kWStride * 2;
 }
 
-cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
+namespace {
+
+template <bool RANKS>
+cudaError_t launch_combine_impl(const DecodeArgs& a, const RankSources& src, cudaStream_t stream) {
   const size_t smem = decode_combine_smem_bytes(a.d_c);
-  cudaError_t e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_combine_kernel<RANKS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   const int T = a.batch * a.nq;
   const int KS = (a.d_c + kSlice - 1) / kSlice;   // d_c <= 512: at most 2
@@ -264,9 +302,20 @@ cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
   attr[1] = pdl_attribute();
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, a, KS);
+  e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<RANKS>, a, src, KS);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream) {
+  RankSources none = {};
+  return launch_combine_impl<false>(a, none, stream);
+}
+
+cudaError_t launch_merge_ranks(const DecodeArgs& a, const RankSources& src, cudaStream_t stream) {
+  return launch_combine_impl<true>(a, src, stream);
 }
 
 }  // namespace mla

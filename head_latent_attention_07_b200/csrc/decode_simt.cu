@@ -39,7 +39,8 @@ decode_split_simt_kernel(DecodeArgs a) {
 
   grid_dependency_wait();
   allow_dependent_launch();   // after the wait: see decode_tc.cu
-  build_plan(&sm->plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.dev_status);
+  build_plan(&sm->plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.dev_status, a.kv_rank,
+             a.kv_ranks);
   const int w = blockIdx.x;
   const int row0 = blockIdx.y * kRows;
   const int chunk = sm->plan.chunk;
@@ -89,7 +90,8 @@ decode_split_simt_kernel(DecodeArgs a) {
       for (int k = 0; k < 8; ++k) acc[r][k] = 0.f;
     __syncthreads();
 
-    for (int pg = f - sb; pg < seg_end - sb; ++pg) {
+    const int w0 = sm->plan.win0[b];   // pages are indexed from the sequence's start
+    for (int pg = f - sb + w0; pg < seg_end - sb + w0; ++pg) {
       const int page_id = a.page_table[(size_t)b * a.max_pages + pg];
       if (page_id < 0 || page_id >= a.num_pages) {  // uniform across the CTA
         if (tid == 0) record_status(a.dev_status, MLA_ERR_RANGE);

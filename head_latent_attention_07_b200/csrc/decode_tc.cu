@@ -113,8 +113,8 @@ struct PieceIter {
     const int sb = ps->start[b];
     const int e = min(f1, ps->start[b + 1]);
     p->b = b;
-    p->pg_begin = f - sb;
-    p->pg_end = e - sb;
+    p->pg_begin = f - sb + ps->win0[b];   // absolute page indices of the sequence
+    p->pg_end = e - sb + ps->win0[b];
     p->id = ps->piece_begin[b] + (w - sb / chunk);
     f = e;
     return true;
@@ -229,7 +229,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
   // whose producers (if any) ran before this kernel's wait returned
   allow_dependent_launch();
   build_plan(plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G,
-             (blockIdx.x == 0 && blockIdx.y == 0) ? status : nullptr);  // ends with __syncthreads
+             (blockIdx.x == 0 && blockIdx.y == 0) ? status : nullptr, a.kv_rank, a.kv_ranks);  // ends with __syncthreads
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised before any remote traffic
   tc_fence_after();

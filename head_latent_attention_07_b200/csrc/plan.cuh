@@ -13,6 +13,11 @@
 //
 // Every CTA rebuilds this schedule from seq_lens in shared memory (two block
 // scans over the batch), so no planning launch and no metadata buffer exist.
+//
+// Context split: with kv_ranks > 1 (one call per rank, e.g. one per GPU) rank r
+// takes only the window [P_b r / R, P_b (r + 1) / R) of sequence b's P_b pages;
+// the schedule above is built over the windows, and page indices stay absolute
+// (win0[b] is added back), so masking and the page table are unchanged.
 #pragma once
 
 #include "common.cuh"
@@ -25,6 +30,7 @@ constexpr int kMinChunk = 4;      // pages: keeps per-piece overhead bounded
 struct PlanSmem {
   int start[kMaxBatch + 1];        // first flat page of each sequence; start[B] = total
   int piece_begin[kMaxBatch + 1];  // first piece of each sequence; piece_begin[B] = #pieces
+  int win0[kMaxBatch];             // first page of each sequence's window
   int chunk;                       // pages per worker
   int warp_tot[32];
 };
@@ -73,16 +79,25 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
   return excl;
 }
 
-// Fills ps->start, ps->piece_begin and ps->chunk for `batch` sequences and G workers.
+// First page of rank r's window over n pages (R ranks): floor(n r / R).
+__device__ __forceinline__ int window_begin(int n, int r, int R) { return (int)(((long long)n * r) / R); }
+
+// Fills ps->start, ps->piece_begin, ps->win0 and ps->chunk for `batch` sequences
+// and G workers, over the windows of rank kv_rank of kv_ranks.
 __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens, int batch, int nq, int max_pages,
-                           int page_size, int G, int32_t* dev_status) {
-  // pass 1: pages per sequence -> start offsets
+                           int page_size, int G, int32_t* dev_status, int kv_rank = 0, int kv_ranks = 1) {
+  // pass 1: pages per sequence (in this rank's window) -> start offsets
   int carry = 0;
   for (int base = 0; base < batch; base += blockDim.x) {
     int b = base + threadIdx.x;
     int v = b < batch ? seq_pages(seq_lens, b, nq, max_pages, page_size,
                                   blockIdx.x == 0 && blockIdx.y == 0 ? dev_status : nullptr)
                       : 0;
+    if (b < batch) {
+      const int p0 = window_begin(v, kv_rank, kv_ranks);
+      ps->win0[b] = p0;
+      v = window_begin(v, kv_rank + 1, kv_ranks) - p0;
+    }
     int tot;
     int ex = block_exclusive_scan(v, ps->warp_tot, &tot);
     if (b < batch) ps->start[b] = carry + ex;

@@ -172,6 +172,53 @@ int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16*
                     int32_t* dev_status, void* stream);
 
 /*
+ * mla_decode_attn_partial - one rank's share of a context-split decode.
+ *
+ * For a sequence too long for one GPU the key range is split over kv_ranks
+ * ranks (one call per rank, normally one rank per GPU): rank r attends over the
+ * pages [P_b r / R, P_b (r + 1) / R) of each sequence's P_b = ceil(seq_lens[b] /
+ * page_size) pages (R = kv_ranks), with the masking of mla_decode_attn (absolute
+ * key indices), and writes its softmax-normalised latent output and log-sum-exp:
+ *   o_lat[b][i][h][:] = sum_{n in window} p_n c_n / sum_{n in window} p_n
+ *   lse[b][i][h]      = log sum_{n in window} exp(s_n)   (-inf for an empty window)
+ * mla_merge_ranks then merges the ranks' results.  This is split-KV across
+ * GPUs: the partials are the only data the ranks exchange (d_c + 1 floats per
+ * query row and rank).  kv_ranks = 1 gives the whole cache.
+ *
+ *   o_lat  device fp32 [batch, nq, H, d_c] (output)
+ *   lse    device fp32 [batch, nq, H] (output)
+ *   other arguments as for mla_decode_attn (no W_UV: it is applied by the merge).
+ * 0 <= kv_rank < kv_ranks, else MLA_ERR_INVALID_ARG.
+ */
+int mla_decode_attn_partial(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
+                            const int32_t* page_table, const int32_t* seq_lens, int32_t batch, int32_t nq,
+                            int32_t max_pages, int32_t num_pages, int32_t kv_rank, int32_t kv_ranks,
+                            void* workspace, size_t ws_bytes, float* o_lat, float* lse, int32_t* dev_status,
+                            void* stream);
+
+/*
+ * mla_merge_ranks - merge the ranks' partials of a context-split decode, then W_UV.
+ *
+ * For each query row (token t, head h), with rank r's partial (o_r, lse_r):
+ *   LSE = log sum_r exp(lse_r),  o_lat = sum_r exp(lse_r - LSE) o_r
+ *   out[t][h] = W_UV,h o_lat,  lse_out[t][h] = LSE
+ * the same log-sum-exp merge as the split-KV combine inside mla_decode_attn.
+ *
+ *   o_lat    host array of n_ranks device pointers, each to fp32 [n_tokens, H, d_c]
+ *   lse      host array of n_ranks device pointers, each to fp32 [n_tokens, H]
+ *   w_uv     device bf16 [H, v_head, d_c]
+ *   out      device bf16 [n_tokens, H, v_head] (output)
+ *   lse_out  device fp32 [n_tokens, H] (output) or NULL
+ * The partials are read with plain loads, once each: a pointer may address this
+ * GPU's memory or a peer GPU's memory mapped into this process (NVLink peer
+ * access), so the exchange between the ranks happens inside this kernel.
+ * 1 <= n_ranks <= 16, n_tokens <= 2^18 (else MLA_ERR_UNSUPPORTED); n_tokens == 0
+ * is a no-op.
+ */
+int mla_merge_ranks(const mla_dims* dims, const float* const* o_lat, const float* const* lse, int32_t n_ranks,
+                    int32_t n_tokens, const mla_bf16* w_uv, mla_bf16* out, float* lse_out, void* stream);
+
+/*
  * mla_decode_attn_noalloc - mla_decode_attn for callers that cannot allocate.
  *
  * The pages describe no such call; it exists for deployment.  Some callers

@@ -151,3 +151,31 @@ def test_query_proj_argument_checks(lib):
     assert call(wuq=FAKE_MIS) == M.MLA_ERR_MISALIGNED
     assert call(T=-1) == M.MLA_ERR_INVALID_ARG
     assert call(T=0, h=None, q=None) == M.MLA_OK                     # empty: no-op
+
+
+def test_context_split_argument_checks(lib):
+    d = v3_dims()
+    part = lambda **kw: lib.mla_decode_attn_partial(
+        ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 2, 1, 4, 8, kw.get("r", 0), kw.get("R", 2), FAKE, 1 << 30,
+        kw.get("o", FAKE), kw.get("l", FAKE), None, None)
+    assert part(r=2) == M.MLA_ERR_INVALID_ARG                      # rank outside [0, R)
+    assert part(r=-1) == M.MLA_ERR_INVALID_ARG
+    assert part(R=0) == M.MLA_ERR_INVALID_ARG
+    assert part(o=None) == M.MLA_ERR_INVALID_ARG
+    assert part(l=None) == M.MLA_ERR_INVALID_ARG
+    assert part(o=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+
+    def merge(n=2, T=4, o=None, l=None, out=FAKE):
+        o = o or [FAKE] * max(n, 1)
+        l = l or [FAKE] * max(n, 1)
+        po = (ctypes.c_void_p * len(o))(*o)
+        pl = (ctypes.c_void_p * len(l))(*l)
+        return lib.mla_merge_ranks(ctypes.byref(d), po, pl, n, T, FAKE, out, None, None)
+    assert merge(n=0) == M.MLA_ERR_INVALID_ARG
+    assert merge(n=17) == M.MLA_ERR_UNSUPPORTED
+    assert merge(T=-1) == M.MLA_ERR_INVALID_ARG
+    assert merge(T=(1 << 18) + 1) == M.MLA_ERR_UNSUPPORTED
+    assert merge(o=[FAKE, None]) == M.MLA_ERR_INVALID_ARG
+    assert merge(l=[FAKE, FAKE_MIS]) == M.MLA_ERR_MISALIGNED
+    assert merge(out=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert merge(T=0) == M.MLA_OK                                   # empty: no-op
