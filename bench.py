@@ -25,7 +25,9 @@ the step's output) and the q-LoRA query path c_Q = W_DQ h, q = W_UQ c_Q
 (mla_query_proj, q_lora_rank 1536), each timed alone after the step (neither is
 part of the step); W_O (235 MB at the V3 shape) is larger than L2, W_DQ + W_UQ
 (97.5 MB) are not, so an L2-sized buffer is rewritten before each timed call of
-the query path.
+the query path.  next_rows.prefill: mla_decode_attn on a chunk of 128 new tokens
+per sequence (2 sequences of 32768, V3 heads), compute-bound, against the bf16
+tensor peak.
 
 --impl reference times the CPU oracle (float64 numpy, absorbed form) on a
 bounded sample of the same workload on the host cores, as the comparison arm.
@@ -314,14 +316,50 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
 
     op = measure_out_proj(M, w, dims, out, dev, stream, args.seed + rank)
     qp = measure_query_proj(M, w, dims, dev, stream, args.seed + rank)
+    pf = measure_prefill(M, w, dims, dev, stream, args.seed + rank)
 
-    ms_total, e2e_ms, dec_ms, op_us, qp_us = max_over_ranks(
-        [ms_total, e2e_ms, float(np.mean(decode_ms)), op["time_us"], qp["time_us"]], dev)
+    ms_total, e2e_ms, dec_ms, op_us, qp_us, pf_us = max_over_ranks(
+        [ms_total, e2e_ms, float(np.mean(decode_ms)), op["time_us"], qp["time_us"], pf["time_us"]], dev)
     op["time_us"] = op_us
     qp["time_us"] = qp_us
+    pf["time_us"] = pf_us
     return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": dec_ms, "clocks": clocks,
             "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens,
-            "out_proj": op, "query_proj": qp}
+            "out_proj": op, "query_proj": qp, "prefill": pf}
+
+
+def measure_prefill(M, w: W.Workload, dims, dev, stream, seed: int, chunk: int = 128, batch: int = 2,
+                    context: int = 32768, iters: int = 5) -> dict:
+    """Average device time of mla_decode_attn on a prefill chunk: `chunk` new tokens
+    per sequence (already appended), each attending causally over its sequence."""
+    import torch
+    wp = dataclasses.replace(w, name="prefill", batch=batch, nq=chunk, context=context)
+    x = W.make_decode_inputs(wp, seed=seed)
+    to_bf16 = lambda b: torch.from_numpy(np.ascontiguousarray(b)).view(torch.bfloat16).to(dev)
+    to_i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+    pool, page_table, lens, pos = to_bf16(x.bits["pool"]), to_i32(x.page_table), to_i32(x.lens), to_i32(x.pos)
+    T = wp.tokens
+    q_lat = torch.empty((batch, chunk, wp.n_heads, wp.row), dtype=torch.bfloat16, device=dev)
+    M.mla_absorb_q(dims, to_bf16(x.bits["q"]), pos, to_bf16(x.bits["w_uk"]), q_lat.view(T, wp.n_heads, wp.row),
+                   stream=stream)
+    w_uv = to_bf16(x.bits["w_uv"])
+    out = torch.empty((batch, chunk, wp.n_heads, wp.v_head), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((batch, chunk, wp.n_heads), dtype=torch.float32, device=dev)
+    ws = torch.empty(M.mla_decode_workspace_bytes(dims, batch, chunk), dtype=torch.uint8, device=dev)
+    call = lambda: M.mla_decode_attn(dims, q_lat, pool, page_table, lens, w_uv, ws, out, lse, stream=stream)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    keys = int(sum(int(n) - chunk + i + 1 for n in x.lens for i in range(chunk)))   # visible keys, all queries
+    flops = keys * wp.n_heads * 2 * (wp.row + wp.d_c) + T * wp.n_heads * 2 * wp.d_c * wp.v_head
+    return {"time_us": e0.elapsed_time(e1) * 1000.0 / iters, "flops": flops, "launches": 2 * iters,
+            "shape": f"{batch} sequences x {chunk} new tokens, context {context}, {wp.n_heads} heads"}
 
 
 def measure_query_proj(M, w: W.Workload, dims, dev, stream, seed: int, iters: int = 50) -> dict:
@@ -526,6 +564,13 @@ def main():
         "shape": qp["shape"], "bound": "hbm", "achieved": qp_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": qp_gbs / peaks["hbm_gbs"], "time_us": qp["time_us"], "bytes_per_call": qp["bytes_per_launch"],
         "launches_timed": qp["launches"], "l2": "256 MB buffer rewritten before each call"}
+    pf = r["prefill"]
+    pf_tfs = pf["flops"] / (pf["time_us"] * 1e-6) / 1e12
+    line["next_rows"]["prefill"] = {
+        "kernel": "mla_decode_attn (split + combine) on a prefill chunk, timed alone after the step",
+        "shape": pf["shape"], "bound": "tensor", "achieved": pf_tfs, "peak": peaks["bf16_tflops"],
+        "unit": "TFLOP/s", "frac": pf_tfs / peaks["bf16_tflops"], "time_us": pf["time_us"],
+        "flops_per_call": pf["flops"], "launches_timed": pf["launches"]}
     if world == 1 and not args.no_cpu_baseline:
         arm = OracleArm(w, args.seed)
         v, sample = arm.measure(args.cpu_budget)

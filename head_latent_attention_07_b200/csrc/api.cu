@@ -12,6 +12,12 @@ constexpr float kDefaultTheta = 10000.f;
 constexpr int32_t kMaxOutProjTokens = 1 << 20;   // tokens of one out / query projection call
 constexpr int32_t kMaxQLoraRank = 1 << 16;
 constexpr int32_t kMaxMergeTokens = 1 << 18;     // grid rows of the rank merge stay below 65536
+// Query tokens per sequence of one decode call: 1 or 2 in decode, up to a
+// chunk of 1024 in chunked prefill; batch * nq is bounded like the merge's tokens.
+constexpr int32_t kMaxNq = 1024;
+bool decode_shape_ok(int32_t batch, int32_t nq) {
+  return batch <= mla::kMaxBatch && nq <= kMaxNq && (int64_t)batch * nq <= kMaxMergeTokens;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -56,9 +62,19 @@ struct WsLayout {
   size_t part_o_bytes, part_lse_bytes, total;
 };
 
-// Workspace for at most (#SMs + batch) split pieces of nq*H rows each.
+// Split workers of a decode call: one CTA pair per worker and 128-row tile on the
+// tensor-core path (fewer workers when there are many row tiles, as in chunked
+// prefill), else a share of two CTAs per SM over the 16-row groups.
+int decode_workers(const mla_dims* d, int nq, int sms) {
+  if (mla::decode_tc_supported(d->d_c, d->d_rope, d->page_size)) return mla::decode_tc_workers(sms, nq * d->n_heads);
+  const int groups = mla::decode_simt_row_groups(nq * d->n_heads);
+  const int G = (2 * sms + groups - 1) / groups;
+  return G < 1 ? 1 : (G > sms ? sms : G);
+}
+
+// Workspace for at most (workers + batch) split pieces of nq*H rows each.
 WsLayout ws_layout(const mla_dims* d, int batch, int nq, int sms) {
-  const size_t pieces = (size_t)mla::max_pieces(sms, batch);
+  const size_t pieces = (size_t)mla::max_pieces(decode_workers(d, nq, sms), batch);
   const size_t rows = (size_t)nq * d->n_heads;
   WsLayout w;
   w.part_o_bytes = align256(pieces * rows * d->d_c * sizeof(float));
@@ -117,7 +133,7 @@ int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
 }
 
 size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t nq) {
-  if (check_dims(dims) != MLA_OK || batch < 1 || batch > mla::kMaxBatch || nq < 1 || nq > 16) return 0;
+  if (check_dims(dims) != MLA_OK || batch < 1 || nq < 1 || !decode_shape_ok(batch, nq)) return 0;
   int sms = 0;
   if (device_sms(&sms) != MLA_OK) return 0;
   return ws_layout(dims, batch, nq, sms).total;
@@ -137,7 +153,7 @@ int decode_common(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* p
   if (st != MLA_OK) return st;
   if (batch < 1 || nq < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
   if (kv_ranks < 1 || kv_rank < 0 || kv_rank >= kv_ranks) return MLA_ERR_INVALID_ARG;
-  if (batch > mla::kMaxBatch || nq > 16) return MLA_ERR_UNSUPPORTED;
+  if (!decode_shape_ok(batch, nq)) return MLA_ERR_UNSUPPORTED;
   if ((int64_t)max_pages * dims->page_size > INT32_MAX) return MLA_ERR_UNSUPPORTED;
   if (!q_lat || !pool || !page_table || !seq_lens || !workspace || (!out && !o_lat)) return MLA_ERR_INVALID_ARG;
   if (out && !w_uv) return MLA_ERR_INVALID_ARG;
@@ -160,14 +176,11 @@ int decode_common(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* p
   a.num_pages = num_pages; a.scale = eff_scale(dims);
   a.kv_rank = kv_rank; a.kv_ranks = kv_ranks;
   cudaStream_t s = (cudaStream_t)stream;
+  a.G = decode_workers(dims, nq, sms);
   if (mla::decode_tc_supported(dims->d_c, dims->d_rope, dims->page_size)) {
     // tensor-core path: one CTA pair per worker and 128-row tile
-    a.G = mla::decode_tc_workers(sms, nq * dims->n_heads);
     if ((st = cuda_status(mla::launch_decode_split_tc(a, mla::kSpinLimitCycles, s))) != MLA_OK) return st;
   } else {
-    const int groups = mla::decode_simt_row_groups(nq * dims->n_heads);
-    int G = (2 * sms + groups - 1) / groups;
-    a.G = G < 1 ? 1 : (G > sms ? sms : G);
     if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
   }
   return cuda_status(mla::launch_decode_combine(a, s));

@@ -163,7 +163,12 @@ size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n
  *   dev_status device int32 word or NULL
  * A sequence whose length is out of range gets zero output and lse = -inf; a
  * page-table entry outside [0, num_pages) is skipped (never read).  Both record
- * MLA_ERR_RANGE in dev_status.  batch <= 1024, nq <= 16.
+ * MLA_ERR_RANGE in dev_status.  batch <= 1024, nq <= 1024, batch * nq <= 2^18
+ * (else MLA_ERR_UNSUPPORTED).  nq > 1 covers decode with several new tokens per
+ * sequence and chunked prefill: a chunk of nq new tokens, appended by
+ * mla_append_latent first, attends causally (token i of the chunk sees the cache
+ * up to its own index).  Each group of 128 query rows (token, head) streams the
+ * sequence's pages once.
  */
 int mla_decode_attn(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* pool,
                     const int32_t* page_table, const int32_t* seq_lens, int32_t batch,

@@ -105,7 +105,8 @@ def test_decode_argument_checks(lib):
     assert call(B=0) == M.MLA_ERR_INVALID_ARG
     assert call(nq=0) == M.MLA_ERR_INVALID_ARG
     assert call(B=1025) == M.MLA_ERR_UNSUPPORTED
-    assert call(nq=17) == M.MLA_ERR_UNSUPPORTED
+    assert call(nq=1025) == M.MLA_ERR_UNSUPPORTED
+    assert call(B=1000, nq=1000) == M.MLA_ERR_UNSUPPORTED     # batch * nq above 2^18
     assert call(mp=1 << 26) == M.MLA_ERR_UNSUPPORTED       # max_pages * page overflows int32
     assert call(out=FAKE_MIS) == M.MLA_ERR_MISALIGNED
     assert call(lse=FAKE + 4) == M.MLA_ERR_MISALIGNED

@@ -93,6 +93,36 @@ def test_ragged_lengths_and_pieces(nq, lens):
     check_step(x, g)
 
 
+@pytest.mark.parametrize("nq,lens", [
+    (32, [32, 40, 300]),       # the first chunk is the whole sequence
+    (64, [64, 65, 1000]),
+    (128, [128, 129, 2000]),
+])
+def test_chunked_prefill(nq, lens):
+    # a chunk of nq new tokens per sequence, appended then attending causally;
+    # absorbed form for every (token, head), naive form on a few pairs
+    w = W.Workload("prefill_small", batch=len(lens), nq=nq, context=None, ragged=(1, 1), **SMALL)
+    x = W.make_decode_inputs(w, seed=50 + nq, lens=lens)
+    g = GpuStep(x).run()
+    assert g.device_status() == 0
+    check_step(x, g, form="absorbed")
+    args = oracle_inputs(x)
+    args["pool"] = Bf16Pool(x.bits["pool"])
+    out = f64_of(g.out).reshape(w.tokens, w.n_heads, w.v_head)
+    for t, h in ((0, 0), (nq - 1, 7), (w.tokens - 1, 3)):
+        ref = O.decode_step(**args, heads=[h], queries=[t])
+        assert_close(out[t, h], ref["out"][t, h], f"out naive ({t},{h})")
+
+
+def test_chunked_prefill_v3_heads_sampled():
+    w = W.Workload("prefill_v3", batch=2, nq=64, n_heads=128, d_model=7168, d_c=512, d_rope=64,
+                   qk_nope=128, v_head=128, context=4096)
+    x = W.make_decode_inputs(w, seed=60)
+    g = GpuStep(x).run()
+    assert g.device_status() == 0
+    check_step(x, g, heads=[0, 64, 127], queries=[0, 31, 63, 64, 100, 127], form="absorbed")
+
+
 def test_decode_only_with_peaked_scores():
     # q_lat drawn directly; some keys planted along q~ so the running max jumps late
     w = W.Workload("peaked", batch=3, nq=1, context=3000, **SMALL)
