@@ -66,7 +66,22 @@ struct WsLayout {
 // tensor-core path (fewer workers when there are many row tiles, as in chunked
 // prefill), else a share of two CTAs per SM over the 16-row groups.
 int decode_workers(const mla_dims* d, int nq, int sms) {
-  if (mla::decode_tc_supported(d->d_c, d->d_rope, d->page_size)) return mla::decode_tc_workers(sms, nq * d->n_heads);
+  if (mla::decode_tc_supported(d->d_c, d->d_rope, d->page_size)) {
+    const int tiles = (nq * d->n_heads + 127) / 128;
+    const int pairs = sms / 2;
+    const int g_decode = mla::decode_tc_workers(sms, nq * d->n_heads);
+    if (g_decode > 1) return g_decode;   // few row tiles (decode): one wave of pairs
+    // many row tiles (chunked prefill): split each tile's pages over G workers,
+    // G <= 8 chosen so that the last wave of CTA pairs is as full as possible
+    int best = 1;
+    double best_fill = 0.0;
+    for (int g = 1; g <= 8; ++g) {
+      const long long units = (long long)tiles * g;
+      const double fill = (double)units / (double)(((units + pairs - 1) / pairs) * pairs);
+      if (fill > best_fill + 1e-9) { best_fill = fill; best = g; }
+    }
+    return best;
+  }
   const int groups = mla::decode_simt_row_groups(nq * d->n_heads);
   const int G = (2 * sms + groups - 1) / groups;
   return G < 1 ? 1 : (G > sms ? sms : G);
