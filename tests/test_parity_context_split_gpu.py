@@ -123,3 +123,25 @@ def test_long_context_four_ranks_full_size_sampled():
     out, lse = run_merge(g, run_partials(g, 4))
     assert g.device_status() == 0
     check_merged(x, g, out, lse, heads=[0, 77, 127])
+
+
+def test_context_split_decode_one_rank_nccl_group(tmp_path):
+    # the package's plumbing on one GPU: a one-rank NCCL group, the gather of one
+    # partial, the merge: bit for bit the one-call result
+    import torch.distributed as dist
+    from head_latent_attention_07_b200.context_split import context_split_decode
+    dist.init_process_group("nccl", init_method=f"file://{tmp_path}/pg", rank=0, world_size=1)
+    try:
+        w = W.Workload("cp_nccl", batch=3, nq=2, context=None, ragged=(1, 1), **SMALL)
+        x = W.make_decode_inputs(w, seed=77, lens=[65, 300, 1000])
+        g = GpuStep(x).run()
+        out = torch.full_like(g.out, float("nan"))
+        lse = torch.full_like(g.lse, float("nan"))
+        context_split_decode(g.dims, g.q_lat.view(w.batch, w.nq, w.n_heads, w.row), g.pool, g.page_table,
+                             g.seq_lens, g.w_uv, g.ws, out, lse, dev_status=g.status)
+        torch.cuda.synchronize()
+        assert torch.equal(out, g.out)
+        assert torch.equal(lse, g.lse)
+        assert g.device_status() == 0
+    finally:
+        dist.destroy_process_group()
