@@ -1,6 +1,7 @@
 // C ABI of libmla_b200.so: argument validation, workspace sizing, launches.
 // The declarations and the contract of every entry point are in include/mla.h.
 #include <math.h>
+#include <stdlib.h>
 
 #include "../../include/mla.h"
 #include "decode.h"
@@ -20,6 +21,19 @@ bool decode_shape_ok(int32_t batch, int32_t nq) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Spin budget of each bounded wait in the split kernel: kSpinLimitCycles, or the
+// environment variable MLA_SPIN_LIMIT (cycles, >= 0) when it is set, which lets a
+// test make the waits run out.
+long long spin_limit_cycles() {
+  const char* e = getenv("MLA_SPIN_LIMIT");
+  if (e != nullptr && *e != 0) {
+    char* end = nullptr;
+    const long long v = strtoll(e, &end, 10);
+    if (end != nullptr && *end == 0 && v >= 0) return v;
+  }
+  return mla::kSpinLimitCycles;
+}
 
 // Shape checks shared by all calls.  d_rope == 0 is refused: without the
 // decoupled RoPE channels W_UK cannot be folded into the query (the rotation
@@ -194,7 +208,7 @@ int decode_common(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* p
   a.G = decode_workers(dims, nq, sms);
   if (mla::decode_tc_supported(dims->d_c, dims->d_rope, dims->page_size)) {
     // tensor-core path: one CTA pair per worker and 128-row tile
-    if ((st = cuda_status(mla::launch_decode_split_tc(a, mla::kSpinLimitCycles, s))) != MLA_OK) return st;
+    if ((st = cuda_status(mla::launch_decode_split_tc(a, spin_limit_cycles(), s))) != MLA_OK) return st;
   } else {
     if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
   }

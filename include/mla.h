@@ -41,6 +41,10 @@
  *     sequence length outside the page table, a bounded wait that ran out) are
  *     recorded, first one wins, in the caller's int32 status word `dev_status`
  *     (may be NULL) and the offending access is skipped: no kernel traps.
+ *   - Bounded waits: each wait between the roles of the decode kernels gives up
+ *     after about 2^31 cycles (~1 s), records MLA_ERR_TIMEOUT and ends the kernel
+ *     cleanly.  The environment variable MLA_SPIN_LIMIT (cycles, read at each
+ *     call) overrides the budget; tests set it small to exercise that path.
  *   - RoPE: channel pair (2i, 2i+1) rotates by pos * theta^(-2i/d_rope), the
  *     angle evaluated in double precision; pos = cache index of the token.
  *   - bf16 outputs are rounded to nearest even from fp32 accumulators.
