@@ -9,9 +9,15 @@ importing the binding fails loudly when the shared library has not been built.
     import head_latent_attention_07_b200 as mla
     dims = mla.MlaDims(n_heads=128, d_c=512, d_rope=64, qk_nope=128, v_head=128,
                        d_model=7168, page_size=64)
+    mla.mla_query_proj(dims, h, w_dq, w_uq, c_q, q)          # q-LoRA query path (optional)
     mla.mla_append_latent(dims, h, w_dkv, seq_idx, pos, page_table, pool)
     mla.mla_absorb_q(dims, q, pos, w_uk, q_lat)
     mla.mla_decode_attn(dims, q_lat, pool, page_table, seq_lens, w_uv, workspace, out, lse)
+    mla.mla_out_proj(dims, out, w_o, y)                       # layer output (optional)
+
+Context split of long sequences over ranks: mla_decode_attn_partial on each
+rank's window, then mla_merge_ranks (see context_split.py for the process-group
+form).
 """
 from __future__ import annotations
 

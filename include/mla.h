@@ -9,7 +9,9 @@
  *                      log-sum-exp combine of the splits, then W_UV
  * Around them: mla_query_proj (the queries from the hidden state through the
  * compressed query latent, before mla_absorb_q) and mla_out_proj (the layer
- * output W_O concat_h(o_h), after mla_decode_attn).
+ * output W_O concat_h(o_h), after mla_decode_attn).  For sequences too long
+ * for one GPU, mla_decode_attn_partial (one rank's window of the pages) and
+ * mla_merge_ranks (the ranks' partials merged, then W_UV) split the key range.
  * Keys and values are never decompressed: every cached token holds only its
  * latent c_t (d_c scalars) and its decoupled RoPE key k_t^R (d_rope scalars).
  *
