@@ -123,6 +123,24 @@ def test_chunked_prefill_v3_heads_sampled():
     check_step(x, g, heads=[0, 64, 127], queries=[0, 31, 63, 64, 100, 127], form="absorbed")
 
 
+def test_output_invariant_under_physical_page_shuffle():
+    # the same logical cache stored under another permutation of the physical
+    # pages: every output bit and every appended row must be the same
+    import dataclasses
+    w = W.Workload("reshuffled", batch=3, nq=2, context=None, ragged=(1, 1), **SMALL)
+    x1 = W.make_decode_inputs(w, seed=13, spare_pages=2, lens=[65, 300, 1000])
+    perm = np.random.default_rng(99).permutation(x1.num_pages).astype(np.int32)
+    pool2 = np.empty_like(x1.bits["pool"])
+    pool2[perm] = x1.bits["pool"]
+    table2 = np.where(x1.page_table >= 0, perm[np.maximum(x1.page_table, 0)], -1).astype(np.int32)
+    x2 = dataclasses.replace(x1, page_table=table2, bits={**x1.bits, "pool": pool2})
+    g1, g2 = GpuStep(x1).run(), GpuStep(x2).run()
+    assert g1.device_status() == 0 and g2.device_status() == 0
+    assert torch.equal(g1.out, g2.out)
+    assert torch.equal(g1.lse, g2.lse)
+    assert np.array_equal(bits_of(g2.pool)[perm], bits_of(g1.pool))
+
+
 def test_decode_only_with_peaked_scores():
     # q_lat drawn directly; some keys planted along q~ so the running max jumps late
     w = W.Workload("peaked", batch=3, nq=1, context=3000, **SMALL)
