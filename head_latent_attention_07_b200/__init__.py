@@ -283,13 +283,17 @@ def mla_merge_ranks(dims: MlaDims, o_lats, lses, w_uv, out, lse=None, stream=Non
     R = len(o_lats)
     if R != len(lses) or R < 1:
         raise ValueError("one o_lat and one lse per rank")
+    if out.dim() < 3 or tuple(out.shape[-2:]) != (dims.n_heads, dims.v_head):
+        raise ValueError(f"out must be [..., {dims.n_heads}, {dims.v_head}], got {tuple(out.shape)}")
     T = out.numel() // (dims.n_heads * dims.v_head)
-    _shape(out.view(T, dims.n_heads, dims.v_head), (T, dims.n_heads, dims.v_head), "out")
+    _shape(w_uv, (dims.n_heads, dims.v_head, dims.d_c), "w_uv")
     for o, l in zip(o_lats, lses):
-        if o.numel() != T * dims.n_heads * dims.d_c or l.numel() != T * dims.n_heads:
-            raise ValueError("partials must be [T, H, d_c] and [T, H]")
-    if lse is not None and lse.numel() != T * dims.n_heads:
-        raise ValueError("lse must hold T * H values")
+        if tuple(o.shape[-2:]) != (dims.n_heads, dims.d_c) or o.numel() != T * dims.n_heads * dims.d_c:
+            raise ValueError(f"each o_lat must be [..., {dims.n_heads}, {dims.d_c}] with T = {T} tokens")
+        if l.shape[-1] != dims.n_heads or l.numel() != T * dims.n_heads:
+            raise ValueError(f"each lse must be [..., {dims.n_heads}] with T = {T} tokens")
+    if lse is not None and (lse.shape[-1] != dims.n_heads or lse.numel() != T * dims.n_heads):
+        raise ValueError(f"lse must be [..., {dims.n_heads}] with T = {T} tokens")
     po = (ctypes.c_void_p * R)(*[_ptr(o, torch.float32, "o_lat").value for o in o_lats])
     pl = (ctypes.c_void_p * R)(*[_ptr(l, torch.float32, "lse").value for l in lses])
     st = load_library().mla_merge_ranks(

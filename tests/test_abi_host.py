@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import head_latent_attention_07_b200 as M
 
@@ -180,3 +181,23 @@ def test_context_split_argument_checks(lib):
     assert merge(l=[FAKE, FAKE_MIS]) == M.MLA_ERR_MISALIGNED
     assert merge(out=FAKE_MIS) == M.MLA_ERR_MISALIGNED
     assert merge(T=0) == M.MLA_OK                                   # empty: no-op
+
+
+def test_merge_binding_rejects_mismatched_shapes():
+    # shape checks in the binding run before any pointer is taken (CPU tensors suffice)
+    d = v3_dims()
+    T, H = 4, d.n_heads
+    o = torch.zeros(T, H, d.d_c)
+    l = torch.zeros(T, H)
+    w_uv = torch.zeros(H, d.v_head, d.d_c, dtype=torch.bfloat16)
+    out = torch.zeros(T, H, d.v_head, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        M.mla_merge_ranks(d, [o], [l, l], w_uv, out)                       # one lse too many
+    with pytest.raises(ValueError):
+        M.mla_merge_ranks(d, [torch.zeros(T, H, d.d_c - 8)], [l], w_uv, out)
+    with pytest.raises(ValueError):
+        M.mla_merge_ranks(d, [o], [torch.zeros(T + 1, H)], w_uv, out)
+    with pytest.raises(ValueError):
+        M.mla_merge_ranks(d, [o], [l], w_uv, torch.zeros(T, H, d.v_head + 8, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        M.mla_merge_ranks(d, [o], [l], w_uv[:, :64], out)
