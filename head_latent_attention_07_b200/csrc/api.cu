@@ -122,6 +122,10 @@ int cuda_status(cudaError_t e) {
 
 }  // namespace
 
+namespace mla {
+int record_cuda_error(cudaError_t e) { return cuda_status(e); }
+}  // namespace mla
+
 extern "C" {
 
 int mla_append_latent(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv,

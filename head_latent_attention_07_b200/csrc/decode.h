@@ -1,6 +1,7 @@
 // Internal interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -80,7 +81,12 @@ cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t stream);
 // LSE merge of the ranks' partials, then W_UV: a.batch = tokens, a.nq = 1.
 cudaError_t launch_merge_ranks(const DecodeArgs& a, const RankSources& src, cudaStream_t stream);
 
-// Tensor-core split kernel (d_c = 512, d_rope = 64, 64-token pages).
+// 2-D TMA map over bf16 rows of 576 elements (row stride 1152 bytes) with a box
+// of [box_rows x box_cols] elements (tma_map.cu).
+bool encode_rows576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                    CUtensorMapSwizzle sw);
+
+// Tensor-core split kernels (d_c = 512, d_rope = 64, 64-token pages).
 bool decode_tc_supported(int d_c, int d_rope, int page_size);
 int decode_tc_workers(int sms, int rows_total);
 cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cudaStream_t stream);
@@ -95,6 +101,10 @@ inline cudaLaunchAttribute pdl_attribute() {
   at.val.programmaticStreamSerializationAllowed = 1;
   return at;
 }
+// MLA_OK for cudaSuccess; otherwise remembers `e` for mla_last_cuda_error (per host
+// thread) and returns MLA_ERR_CUDA (api.cu).
+int record_cuda_error(cudaError_t e);
+
 cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
 int linear_ksplit(int N, int K, int sms);

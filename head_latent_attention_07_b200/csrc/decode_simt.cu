@@ -90,7 +90,7 @@ decode_split_simt_kernel(DecodeArgs a) {
       for (int k = 0; k < 8; ++k) acc[r][k] = 0.f;
     __syncthreads();
 
-    const int w0 = sm->plan.win0[b];   // pages are indexed from the sequence's start
+    const int w0 = plan_win0(&sm->plan, b);   // pages are indexed from the sequence's start
     for (int pg = f - sb + w0; pg < seg_end - sb + w0; ++pg) {
       const int page_id = a.page_table[(size_t)b * a.max_pages + pg];
       if (page_id < 0 || page_id >= a.num_pages) {  // uniform across the CTA

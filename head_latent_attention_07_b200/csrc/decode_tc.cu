@@ -91,36 +91,6 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= kNumBars * 8, "barrier area");
 
-// One (sequence, page range) overlap of this worker's chunk.
-struct Piece {
-  int b, pg_begin, pg_end, id;
-};
-
-// Iterates the pieces of worker w in order; identical in every role.
-struct PieceIter {
-  const PlanSmem* ps;
-  int batch, w, chunk, f, f1, b;
-  __device__ PieceIter(const PlanSmem* ps_, int batch_, int w_) : ps(ps_), batch(batch_), w(w_) {
-    chunk = ps->chunk;
-    const int total = ps->start[batch];
-    f = w * chunk;
-    f1 = min(f + chunk, total);
-    b = f < f1 ? seq_of_flat_page(ps, batch, f) : 0;
-  }
-  __device__ bool next(Piece* p) {
-    if (f >= f1) return false;
-    while (ps->start[b + 1] <= f) ++b;
-    const int sb = ps->start[b];
-    const int e = min(f1, ps->start[b + 1]);
-    p->b = b;
-    p->pg_begin = f - sb + ps->win0[b];   // absolute page indices of the sequence
-    p->pg_end = e - sb + ps->win0[b];
-    p->id = ps->piece_begin[b] + (w - sb / chunk);
-    f = e;
-    return true;
-  }
-};
-
 // Walks the pages of worker w: jj counts pages across pieces, p counts pieces.
 struct PageCursor {
   PieceIter it;
@@ -147,6 +117,13 @@ struct PageCursor {
   __device__ bool first() const { return pg == pc.pg_begin; }
   __device__ bool last() const { return pg == pc.pg_end - 1; }
 };
+
+// One lane of the (converged) warp returns true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t is_leader;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(is_leader));
+  return is_leader != 0;
+}
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
@@ -288,54 +265,83 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
     // ------------------------------------------------------------ MMA issuer
     // Two in-order queues, each issued as soon as its inputs are ready: GEMM1
     // (scores, up to two pages ahead: S is double-buffered) and GEMM2 (values,
-    // checked first).
-    if (lane == 0) {
+    // checked first).  The whole warp runs the loop: lane 0 tests the barriers and
+    // walks the pages, the other lanes follow its decision word (broadcast by
+    // shuffle), so that the MMA operands stay warp-uniform, and one elected lane
+    // issues.  (Issued from a lone lane under data-dependent control flow, each MMA
+    // cost several times its execution time on B200.)
+    {
+      constexpr uint32_t kGo1 = 1, kGo2 = 2, kFirst2 = 4, kLast1 = 8, kStop = 16;
       const uint32_t id1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id2 = idesc_bf16_f32(128, 256, 0, 1);
       const uint32_t qra = smem_u32(qr_s);
       PageCursor g1(plan, a.batch, w), g2(plan, a.batch, w);
-      bool has1 = g1.next(), has2 = g2.next();
-      bool q_ok = false;  // query tile of g1's piece is resident
-      int last2 = -1;     // last page whose value MMAs were issued
+      bool has1 = false, has2 = false;
+      if (lane == 0) {
+        has1 = g1.next();
+        has2 = g2.next();
+      }
+      bool q_ok = false;       // query tile of g1's piece is resident (lane 0)
+      int jj1 = 0, jj2 = 0;    // pages issued by the two queues (all lanes)
       long long t_last = clock64();
-      while (has1 || has2) {
-        bool progressed = false;
-        if (has2 && (!has1 || g2.jj < g1.jj)) {
-          const int jj = g2.jj;
-          const bool first = g2.first();
-          const bool ready = (!(first && g2.p > 0) || mbar_test(&bar->o_free, (g2.p - 1) & 1)) &&
-                             mbar_test(&bar->p_full[jj & 1], (jj >> 1) & 1);
-          if (ready) {
+      while (true) {
+        uint32_t word = 0;
+        if (lane == 0) {
+          if (!has1 && !has2) {
+            word = kStop;
+          } else {
+            if (has2 && (!has1 || g2.jj < g1.jj)) {
+              const bool first = g2.first();
+              if ((!(first && g2.p > 0) || mbar_test(&bar->o_free, (g2.p - 1) & 1)) &&
+                  mbar_test(&bar->p_full[g2.jj & 1], (g2.jj >> 1) & 1))
+                word |= kGo2 | (first ? kFirst2 : 0);
+            }
+            if (has1) {
+              const int jj = g1.jj;
+              if (g1.first() && !q_ok) q_ok = mbar_test(&bar->q_full, g1.p & 1);
+              if ((!g1.first() || q_ok) && (jj < 2 || mbar_test(&bar->s_empty[jj & 1], ((jj >> 1) - 1) & 1)) &&
+                  mbar_test(&bar->pg_full[jj % kStages], (jj / kStages) & 1))
+                word |= kGo1 | (g1.last() ? kLast1 : 0);
+            }
+            if (word & (kGo1 | kGo2)) {
+              t_last = clock64();
+            } else if (*abort_flag) {
+              word = kStop;
+            } else if (clock64() - t_last > lim) {
+              record_status(status, MLA_ERR_TIMEOUT);
+              *abort_flag = 1;
+              word = kStop;
+            }
+          }
+        }
+        word = __shfl_sync(0xffffffffu, word, 0);
+        if (word & kStop) break;
+        if (word & kGo2) {
+          const uint32_t pa = smem_u32(p_s + (jj2 & 1) * kPBytes);
+          const uint32_t pb = smem_u32(pg_s + (jj2 % kStages) * kPageBytes);
+          if (elect_one()) {
             fence_proxy_async_smem();  // P written by threads of both CTAs, read by the tensor core
             tc_fence_after();
-            const uint32_t pa = smem_u32(p_s + (jj & 1) * kPBytes);
-            const uint32_t pb = smem_u32(pg_s + (jj % kStages) * kPageBytes);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t da = smem_desc(pa + ks * 32, 16, 1024, kSwizzle128);
               const uint64_t db = smem_desc(pb + ks * 2048, 8192, 1024, kSwizzle128);
-              mma_bf16(tmem, da, db, id2, (first && ks == 0) ? 0u : 1u);
+              mma_bf16(tmem, da, db, id2, ((word & kFirst2) && ks == 0) ? 0u : 1u);
             }
-            mma_commit(&bar->pg_empty[jj % kStages]);
-            mma_commit(&bar->o_done[jj & 1]);
-            // this CTA's P tile (jj & 1) has been read: the peer may write page jj + 2's half
-            mma_commit_mc(&bar->p_free[jj & 1], uint16_t(1u << peer));
-            last2 = jj;
-            has2 = g2.next();
-            progressed = true;
+            mma_commit(&bar->pg_empty[jj2 % kStages]);
+            mma_commit(&bar->o_done[jj2 & 1]);
+            // this CTA's P tile (jj2 & 1) has been read: the peer may write page jj2 + 2's half
+            mma_commit_mc(&bar->p_free[jj2 & 1], uint16_t(1u << peer));
           }
+          __syncwarp();
+          if (lane == 0) has2 = g2.next();
+          ++jj2;
         }
-        if (has1) {
-          const int jj = g1.jj;
-          const int st = jj % kStages;
-          if (g1.first() && !q_ok) q_ok = mbar_test(&bar->q_full, g1.p & 1);
-          const bool ready = (!g1.first() || q_ok) &&
-                             (jj < 2 || mbar_test(&bar->s_empty[jj & 1], ((jj >> 1) - 1) & 1)) &&
-                             mbar_test(&bar->pg_full[st], (jj / kStages) & 1);
-          if (ready) {
+        if (word & kGo1) {
+          const uint32_t pb = smem_u32(pg_s + (jj1 % kStages) * kPageBytes);
+          const uint32_t ts = tmem + kTmemS + 64 * (jj1 & 1);
+          if (elect_one()) {
             tc_fence_after();
-            const uint32_t pb = smem_u32(pg_s + st * kPageBytes);
-            const uint32_t ts = tmem + kTmemS + 64 * (jj & 1);
 #pragma unroll
             for (int ks = 0; ks < 16; ++ks) {          // latent part: A from TMEM
               const uint64_t db = smem_desc(pb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSwizzle128);
@@ -347,33 +353,30 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
               const uint64_t db = smem_desc(pb + 32768 + ks * 32, 16, 512, kSwizzle64);
               mma_bf16(ts, da, db, id1, 1u);
             }
-            mma_commit(&bar->s_full[jj & 1]);
-            if (g1.last()) {
-              mma_commit(&bar->q_empty);
-              q_ok = false;
-            }
-            has1 = g1.next();
-            progressed = true;
+            mma_commit(&bar->s_full[jj1 & 1]);
+            if (word & kLast1) mma_commit(&bar->q_empty);
           }
-        }
-        if (progressed) {
-          t_last = clock64();
-        } else if (*abort_flag) {
-          break;
-        } else if (clock64() - t_last > lim) {
-          record_status(status, MLA_ERR_TIMEOUT);
-          *abort_flag = 1;
-          break;
+          __syncwarp();
+          if (lane == 0) {
+            if (word & kLast1) q_ok = false;
+            has1 = g1.next();
+          }
+          ++jj1;
         }
       }
       // drain: every MMA issued above has completed before TMEM / smem go away
-      mma_commit(&bar->drain);
-      mbar_wait_drain(&bar->drain, 0, lim);
-      // the peer's value MMAs of the last two pages release this CTA's P tiles by
-      // a multicast arrive that nothing else waits for: let it land
-      const long long lim_drain = *abort_flag ? (1ll << 20) : lim;
-      for (int jj = max(0, last2 - 1); jj <= last2; ++jj)
-        mbar_wait_drain(&bar->p_free[jj & 1], (jj >> 1) & 1, lim_drain);
+      if (elect_one()) mma_commit(&bar->drain);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_wait_drain(&bar->drain, 0, lim);
+        // the peer's value MMAs of the last two pages release this CTA's P tiles by
+        // a multicast arrive that nothing else waits for: let it land
+        const long long lim_drain = *abort_flag ? (1ll << 20) : lim;
+        const int last2 = jj2 - 1;
+        for (int jj = max(0, last2 - 1); jj <= last2; ++jj)
+          mbar_wait_drain(&bar->p_free[jj & 1], (jj >> 1) & 1, lim_drain);
+      }
+      __syncwarp();
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ sender warps
@@ -655,37 +658,6 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
 }
 
 // ------------------------------------------------------------------ host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 map over [rows, 576] with row stride 1152 bytes, box [box_rows, box_cols].
-bool encode_rows576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
-                    CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {576, rows};
-  cuuint64_t strides[1] = {576 * 2};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 }  // namespace
 

@@ -17,7 +17,7 @@
 // Context split: with kv_ranks > 1 (one call per rank, e.g. one per GPU) rank r
 // takes only the window [P_b r / R, P_b (r + 1) / R) of sequence b's P_b pages;
 // the schedule above is built over the windows, and page indices stay absolute
-// (win0[b] is added back), so masking and the page table are unchanged.
+// (the window's first page is added back), so masking and the page table are unchanged.
 #pragma once
 
 #include "common.cuh"
@@ -30,8 +30,10 @@ constexpr int kMinChunk = 4;      // pages: keeps per-piece overhead bounded
 struct PlanSmem {
   int start[kMaxBatch + 1];        // first flat page of each sequence; start[B] = total
   int piece_begin[kMaxBatch + 1];  // first piece of each sequence; piece_begin[B] = #pieces
-  int win0[kMaxBatch];             // first page of each sequence's window
   int chunk;                       // pages per worker
+  // what the window of a sequence is computed from (see plan_win0)
+  const int32_t* seq_lens;
+  int nq, max_pages, page_size, kv_rank, kv_ranks;
   int warp_tot[32];
 };
 
@@ -82,7 +84,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
 // First page of rank r's window over n pages (R ranks): floor(n r / R).
 __device__ __forceinline__ int window_begin(int n, int r, int R) { return (int)(((long long)n * r) / R); }
 
-// Fills ps->start, ps->piece_begin, ps->win0 and ps->chunk for `batch` sequences
+// First page of sequence b's window (0 without a context split).
+__device__ __forceinline__ int plan_win0(const PlanSmem* ps, int b) {
+  if (ps->kv_ranks == 1) return 0;
+  const int len = ps->seq_lens[b];
+  const int pages = (len < ps->nq || len > ps->max_pages * ps->page_size) ? 0 : (len + ps->page_size - 1) / ps->page_size;
+  return window_begin(pages, ps->kv_rank, ps->kv_ranks);
+}
+
+// Fills ps->start, ps->piece_begin, ps->chunk and the window parameters for `batch` sequences
 // and G workers, over the windows of rank kv_rank of kv_ranks.
 __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens, int batch, int nq, int max_pages,
                            int page_size, int G, int32_t* dev_status, int kv_rank = 0, int kv_ranks = 1) {
@@ -93,11 +103,7 @@ __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens
     int v = b < batch ? seq_pages(seq_lens, b, nq, max_pages, page_size,
                                   blockIdx.x == 0 && blockIdx.y == 0 ? dev_status : nullptr)
                       : 0;
-    if (b < batch) {
-      const int p0 = window_begin(v, kv_rank, kv_ranks);
-      ps->win0[b] = p0;
-      v = window_begin(v, kv_rank + 1, kv_ranks) - p0;
-    }
+    if (b < batch) v = window_begin(v, kv_rank + 1, kv_ranks) - window_begin(v, kv_rank, kv_ranks);
     int tot;
     int ex = block_exclusive_scan(v, ps->warp_tot, &tot);
     if (b < batch) ps->start[b] = carry + ex;
@@ -107,6 +113,12 @@ __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens
     ps->start[batch] = carry;
     int c = (carry + G - 1) / G;
     ps->chunk = c < kMinChunk ? kMinChunk : c;
+    ps->seq_lens = seq_lens;
+    ps->nq = nq;
+    ps->max_pages = max_pages;
+    ps->page_size = page_size;
+    ps->kv_rank = kv_rank;
+    ps->kv_ranks = kv_ranks;
   }
   __syncthreads();
   const int chunk = ps->chunk;
@@ -137,5 +149,36 @@ __device__ __forceinline__ int seq_of_flat_page(const PlanSmem* ps, int batch, i
   }
   return lo;  // the largest such b, so empty sequences sharing its start are skipped
 }
+
+// One (sequence, page range) overlap of this worker's chunk.
+struct Piece {
+  int b, pg_begin, pg_end, id;
+};
+
+// Iterates the pieces of worker w in order; identical in every role.
+struct PieceIter {
+  const PlanSmem* ps;
+  int batch, w, chunk, f, f1, b;
+  __device__ PieceIter(const PlanSmem* ps_, int batch_, int w_) : ps(ps_), batch(batch_), w(w_) {
+    chunk = ps->chunk;
+    const int total = ps->start[batch];
+    f = w * chunk;
+    f1 = min(f + chunk, total);
+    b = f < f1 ? seq_of_flat_page(ps, batch, f) : 0;
+  }
+  __device__ bool next(Piece* p) {
+    if (f >= f1) return false;
+    while (ps->start[b + 1] <= f) ++b;
+    const int sb = ps->start[b];
+    const int e = min(f1, ps->start[b + 1]);
+    const int w0 = plan_win0(ps, b);
+    p->b = b;
+    p->pg_begin = f - sb + w0;   // absolute page indices of the sequence
+    p->pg_end = e - sb + w0;
+    p->id = ps->piece_begin[b] + (w - sb / chunk);
+    f = e;
+    return true;
+  }
+};
 
 }  // namespace mla
