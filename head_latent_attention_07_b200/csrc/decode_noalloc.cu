@@ -19,6 +19,8 @@
 #include "../../include/mla.h"
 #include <cuda_runtime.h>
 
+#include "decode.h"
+
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per device
@@ -29,21 +31,25 @@ __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 std::once_flag g_setup_once[kMaxDevices];
 void* g_scratch_addr[kMaxDevices];
-int g_setup_status[kMaxDevices];
+cudaError_t g_setup_error[kMaxDevices];   // outcome of the look-up, reported again on every later call
 
 // Device address of g_decode_scratch on the current device (set-up on first use).
+// A failed look-up is remembered for the device and reported (MLA_ERR_CUDA, with
+// the CUDA error for mla_last_cuda_error) by every later call on it.
 int scratch_on_current_device(void** addr) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  const cudaError_t eg = cudaGetDevice(&dev);
+  if (eg != cudaSuccess) return mla::record_cuda_error(eg);
   if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
   std::call_once(g_setup_once[dev], [dev] {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e == cudaSuccess && p == nullptr) e = cudaErrorInvalidSymbol;
     g_scratch_addr[dev] = (e == cudaSuccess) ? p : nullptr;
-    g_setup_status[dev] = (e == cudaSuccess && p != nullptr) ? MLA_OK : MLA_ERR_CUDA;
+    g_setup_error[dev] = e;
   });
   *addr = g_scratch_addr[dev];
-  return g_setup_status[dev];
+  return mla::record_cuda_error(g_setup_error[dev]);
 }
 
 }  // namespace
