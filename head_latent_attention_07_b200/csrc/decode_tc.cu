@@ -11,7 +11,7 @@
 //           this CTA's columns (latent part of Q_c in TMEM, RoPE part and the page
 //           in shared memory)
 //   swap    CTA c owns the softmax of keys [32c, 32c + 32) of every row: it sends
-//           the peer the partial scores of the peer's keys (fp16, log2 units) and
+//           the peer the partial scores of the peer's keys (fp32, log2 units) and
 //           adds the peer's partials of its own keys to its fp32 ones
 //   softmax the two CTAs agree on each row's running max (one float per row each
 //           way); each computes P (bf16) for its 32 keys and writes it into both
@@ -52,15 +52,16 @@ constexpr int kThreads = 320;  // producer, MMA, 4 sender warps, 4 softmax warps
 constexpr int kStages = 4;
 constexpr int kQrBytes = 128 * 64;            // RoPE block of the query tile [128 x 32] (64-byte swizzle)
 constexpr int kPageBytes = 4 * 8192 + 4096;   // 4 latent blocks [64 x 64] + RoPE block [64 x 32]
-constexpr int kXBytes = 128 * 64;             // received partial scores: [128 rows x 32 keys] fp16
+constexpr int kXBytes = 128 * 128;            // received partial scores: [128 rows x 32 keys] fp32
 constexpr int kPBytes = 128 * 128;            // P tile [128 rows x 64 keys] bf16, 128-byte swizzle
+constexpr int kPTiles = 2;                    // P of pages k, k + 1 in flight
 constexpr int kOffQr = 0;
 constexpr int kOffPg = kOffQr + kQrBytes;
 constexpr int kOffX = kOffPg + kStages * kPageBytes;
 constexpr int kOffP = kOffX + 2 * kXBytes;
-constexpr int kOffM = kOffP + 2 * kPBytes;    // received row maxima [2][128], row sums [128] (fp32)
+constexpr int kOffM = kOffP + kPTiles * kPBytes;  // received row maxima [2][128], row sums [128] (fp32)
 constexpr int kOffPlan = kOffM + 3 * 128 * 4;
-constexpr int kOffBar = kOffPlan + ((int(sizeof(PlanSmem)) + 127) & ~127);
+constexpr int kOffBar = kOffPlan + ((int(sizeof(PlanSmem)) + 15) & ~15);
 constexpr int kNumBars = 32;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;       // TMEM base, abort flag, page metadata
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;       // + 1 KB alignment slack
@@ -85,8 +86,8 @@ struct Bars {
   uint64_t s_full[2], s_empty[2];
   uint64_t x_full[2], x_free[2];   // partial scores from the peer / the peer's slot is free
   uint64_t m_full[2];              // the peer's row maxima of a page
-  uint64_t p_full[2], p_free[2];   // P tile complete (own + peer half) / the peer's P tile is free
-  uint64_t o_done[2];
+  uint64_t p_full[kPTiles], p_free[kPTiles];  // P tile complete (own + peer half) / the peer's P tile is free
+  uint64_t o_done[kPTiles];        // this CTA's value MMAs of the page that used the tile are done
   uint64_t l_full, o_free, drain;
 };
 static_assert(sizeof(Bars) <= kNumBars * 8, "barrier area");
@@ -125,25 +126,11 @@ __device__ __forceinline__ bool elect_one() {
   return is_leader != 0;
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 __device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// fp16 pair -> two fp32 values scaled by 2^-112 (exact for normal and zero
-// halves, sign kept), on the integer pipe: f = bits(x_fp16) re-based as fp32.
-// Multiplying by 2^112 restores the value.
-__device__ __forceinline__ float h_lo_scaled(uint32_t v) {
-  return __uint_as_float(((v & 0x8000u) << 16) | ((v & 0x7FFFu) << 13));
-}
-__device__ __forceinline__ float h_hi_scaled(uint32_t v) {
-  return __uint_as_float((v & 0x80000000u) | ((v >> 3) & 0x0FFFE000u));
-}
-constexpr float kTwo112 = 5.192296858534828e33f;  // 2^112
 
 __global__ void __launch_bounds__(kThreads, 1)
 decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_constant__ CUtensorMap tp128,
@@ -183,6 +170,8 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
       mbar_init(&bar->x_full[s], 1);   // local softmax leader's expect-bytes arrival; the peer's stores carry the bytes
       mbar_init(&bar->x_free[s], 4);   // the peer's 4 softmax warps have read their slot
       mbar_init(&bar->m_full[s], 1);
+    }
+    for (int s = 0; s < kPTiles; ++s) {
       mbar_init(&bar->p_full[s], 4);   // 4 local softmax warps (one also expects the peer's bytes)
       mbar_init(&bar->p_free[s], 1);   // the peer's value MMA of the page has read its P tile
       mbar_init(&bar->o_done[s], 1);
@@ -293,7 +282,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
             if (has2 && (!has1 || g2.jj < g1.jj)) {
               const bool first = g2.first();
               if ((!(first && g2.p > 0) || mbar_test(&bar->o_free, (g2.p - 1) & 1)) &&
-                  mbar_test(&bar->p_full[g2.jj & 1], (g2.jj >> 1) & 1))
+                  mbar_test(&bar->p_full[g2.jj % kPTiles], (g2.jj / kPTiles) & 1))
                 word |= kGo2 | (first ? kFirst2 : 0);
             }
             if (has1) {
@@ -317,7 +306,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
         word = __shfl_sync(0xffffffffu, word, 0);
         if (word & kStop) break;
         if (word & kGo2) {
-          const uint32_t pa = smem_u32(p_s + (jj2 & 1) * kPBytes);
+          const uint32_t pa = smem_u32(p_s + (jj2 % kPTiles) * kPBytes);
           const uint32_t pb = smem_u32(pg_s + (jj2 % kStages) * kPageBytes);
           if (elect_one()) {
             fence_proxy_async_smem();  // P written by threads of both CTAs, read by the tensor core
@@ -329,9 +318,9 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
               mma_bf16(tmem, da, db, id2, ((word & kFirst2) && ks == 0) ? 0u : 1u);
             }
             mma_commit(&bar->pg_empty[jj2 % kStages]);
-            mma_commit(&bar->o_done[jj2 & 1]);
-            // this CTA's P tile (jj2 & 1) has been read: the peer may write page jj2 + 2's half
-            mma_commit_mc(&bar->p_free[jj2 & 1], uint16_t(1u << peer));
+            mma_commit(&bar->o_done[jj2 % kPTiles]);
+            // this CTA's P tile has been read: the peer may write page jj2 + kPTiles's half
+            mma_commit_mc(&bar->p_free[jj2 % kPTiles], uint16_t(1u << peer));
           }
           __syncwarp();
           if (lane == 0) has2 = g2.next();
@@ -369,12 +358,12 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
       __syncwarp();
       if (lane == 0) {
         mbar_wait_drain(&bar->drain, 0, lim);
-        // the peer's value MMAs of the last two pages release this CTA's P tiles by
-        // a multicast arrive that nothing else waits for: let it land
+        // the peer's value MMAs of the last kPTiles pages release this CTA's P tiles
+        // by a multicast arrive that nothing else waits for: let it land
         const long long lim_drain = *abort_flag ? (1ll << 20) : lim;
         const int last2 = jj2 - 1;
-        for (int jj = max(0, last2 - 1); jj <= last2; ++jj)
-          mbar_wait_drain(&bar->p_free[jj & 1], (jj >> 1) & 1, lim_drain);
+        for (int jj = max(0, last2 - (kPTiles - 1)); jj <= last2; ++jj)
+          mbar_wait_drain(&bar->p_free[jj % kPTiles], (jj / kPTiles) & 1, lim_drain);
       }
       __syncwarp();
     }
@@ -388,7 +377,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t x_peer = mapa(smem_u32(x_s), peer);
     const uint32_t xfull_peer = mapa(smem_u32(&bar->x_full[0]), peer);
-    const uint32_t sw = uint32_t((r >> 1) & 3);        // chunk swizzle of row r in a receive slot
+    const uint32_t sw = uint32_t(r & 7);               // chunk swizzle of row r in a receive slot
     auto wwait = [&](uint64_t* b, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, status, lim));
     };
@@ -424,15 +413,18 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->s_empty[slot]);
-      uint32_t h[16];
+      // fp32 in log2 units: a half of the dot product can be large while the whole
+      // score is not (opposite halves), and only fp32 keeps the sum's absolute error
+      // small enough for the softmax weights
+      uint32_t h[32];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) h[i] = pack_half2(sv[2 * i] * prm.scale_log2, sv[2 * i + 1] * prm.scale_log2);
+      for (int i = 0; i < 32; ++i) h[i] = __float_as_uint(sv[i] * prm.scale_log2);
       // the peer's receive slot is free once its softmax warps have read page jj - 2
       if (jj >= 2 && !wwait(&bar->x_free[slot], ((jj >> 1) - 1) & 1)) break;
-      const uint32_t dst = x_peer + slot * kXBytes + r * 64;
+      const uint32_t dst = x_peer + slot * kXBytes + r * 128;
       const uint32_t rbar = xfull_peer + slot * 8;
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4)
+      for (int k4 = 0; k4 < 8; ++k4)
         st_async_v4(dst + ((k4 ^ sw) << 4), make_uint4(h[4 * k4], h[4 * k4 + 1], h[4 * k4 + 2], h[4 * k4 + 3]),
                     rbar);
       last_jj = jj;
@@ -457,8 +449,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
     const bool row_valid = r < rows_valid;
     const int qi = (row0 + r) / a.n_heads;             // query token of this row
     const int ltid = threadIdx.x - 192;                // 0..127
-    const float own_scale = prm.scale_log2 * (1.0f / kTwo112);  // own partial in the peer's 2^-112 units
-    const uint32_t sw = uint32_t((r >> 1) & 3);
+    const uint32_t sw = uint32_t(r & 7);
     const uint32_t xfree_peer = mapa(smem_u32(&bar->x_free[0]), peer);
     const uint32_t mrecv_peer = mapa(smem_u32(m_recv), peer);
     const uint32_t mfull_peer = mapa(smem_u32(&bar->m_full[0]), peer);
@@ -501,17 +492,14 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
       // posted by the consumer, once the slot's previous phase has completed
       if (leader) mbar_arrive_expect_tx(&bar->x_full[slot], kXBytes);
       if (!wwait(&bar->x_full[slot], (jj >> 1) & 1)) { ok = false; break; }
-      const unsigned char* xrow = x_s + slot * kXBytes + r * 64;
+      const unsigned char* xrow = x_s + slot * kXBytes + r * 128;
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {                 // scores carry a factor 2^-112 here
-        const uint4 v = *reinterpret_cast<const uint4*>(xrow + ((k4 ^ sw) << 4));
-        const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i0 = 8 * k4 + 2 * e;
-          s[i0] = fmaf(s[i0], own_scale, h_lo_scaled(pv[e]));
-          s[i0 + 1] = fmaf(s[i0 + 1], own_scale, h_hi_scaled(pv[e]));
-        }
+      for (int k4 = 0; k4 < 8; ++k4) {                 // whole scores in log2 units
+        const float4 v = *reinterpret_cast<const float4*>(xrow + ((k4 ^ sw) << 4));
+        s[4 * k4] = fmaf(s[4 * k4], prm.scale_log2, v.x);
+        s[4 * k4 + 1] = fmaf(s[4 * k4 + 1], prm.scale_log2, v.y);
+        s[4 * k4 + 2] = fmaf(s[4 * k4 + 2], prm.scale_log2, v.z);
+        s[4 * k4 + 3] = fmaf(s[4 * k4 + 3], prm.scale_log2, v.w);
       }
       // the peer may refill this slot: the loads above have returned (their values
       // are consumed), so the arrive needs no release ordering
@@ -530,7 +518,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
         for (int n = 4; n > 0; n >>= 1)
 #pragma unroll
           for (int i = 0; i < n; ++i) t[i] = fmaxf(t[i], t[i + n]);
-        mx = t[0] * kTwo112;
+        mx = t[0];
       }
       // swap the row maxima of the two key halves with the peer
       if (leader) mbar_arrive_expect_tx(&bar->m_full[slot], 128 * 4);
@@ -544,7 +532,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
       if (__any_sync(0xffffffffu, grow && !cb.first() && m_used != -INFINITY)) {
         const float alpha = (grow && m_used != -INFINITY) ? ex2(m_used - m_new) : 1.f;
         const int jp = jj - 1;  // O must hold every earlier page of this piece
-        if (!wwait(&bar->o_done[jp & 1], (jp >> 1) & 1)) { ok = false; break; }
+        if (!wwait(&bar->o_done[jp % kPTiles], (jp / kPTiles) & 1)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 256; cc += 32) {
@@ -566,27 +554,28 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
       for (int i = 0; i < 4; ++i) ps[i] = 0.f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float p0 = ex2(fmaf(s[2 * i], kTwo112, -m_ref));   // ex2(-inf) = 0
-        const float p1 = ex2(fmaf(s[2 * i + 1], kTwo112, -m_ref));
+        const float p0 = ex2(s[2 * i] - m_ref);         // ex2(-inf) = 0
+        const float p1 = ex2(s[2 * i + 1] - m_ref);
         ps[i & 3] += p0 + p1;
         pk[i] = pack_bf162(p0, p1);
       }
       l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      // P(k) -> P tile (k & 1) of both CTAs, keys [32c, 32c + 32) of row r, once
-      // the value MMAs of page k - 2 (own and peer) have read those tiles
-      if (jj >= 2) {
-        if (!wwait(&bar->o_done[slot], ((jj >> 1) - 1) & 1)) { ok = false; break; }
-        if (!wwait(&bar->p_free[slot], ((jj >> 1) - 1) & 1)) { ok = false; break; }
+      // P(k) -> P tile (k mod 3) of both CTAs, keys [32c, 32c + 32) of row r, once
+      // the value MMAs of page k - 3 (own and peer) have read those tiles
+      const int pt = jj % kPTiles;
+      if (jj >= kPTiles) {
+        if (!wwait(&bar->o_done[pt], ((jj / kPTiles) - 1) & 1)) { ok = false; break; }
+        if (!wwait(&bar->p_free[pt], ((jj / kPTiles) - 1) & 1)) { ok = false; break; }
       }
       {
-        const uint32_t prow = slot * kPBytes + r * 128;
+        const uint32_t prow = pt * kPBytes + r * 128;
         unsigned char* own = p_s + prow;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const uint32_t off = ((4 * c + k4) ^ (r & 7)) << 4;   // 128-byte swizzle of the UMMA K-major tile
           const uint4 v = make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
           *reinterpret_cast<uint4*>(own + off) = v;
-          st_async_v4(p_peer + prow + off, v, pfull_peer + slot * 8);
+          st_async_v4(p_peer + prow + off, v, pfull_peer + pt * 8);
         }
       }
       // cache slots past the sequence (or a page never loaded) feed the value
@@ -603,8 +592,8 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (warp == 6) mbar_arrive_expect_tx(&bar->p_full[slot], kPBytes / 2);  // the peer's half
-        else mbar_arrive(&bar->p_full[slot]);
+        if (warp == 6) mbar_arrive_expect_tx(&bar->p_full[pt], kPBytes / 2);  // the peer's half
+        else mbar_arrive(&bar->p_full[pt]);
       }
 
       if (cb.last()) {
@@ -613,7 +602,7 @@ decode_split_tc_kernel(const __grid_constant__ CUtensorMap tq64, const __grid_co
         st_async_b32(lrecv_peer + r * 4, __float_as_uint(l), lfull_peer);
         if (!wwait(&bar->l_full, cb.p & 1)) { ok = false; break; }
         const float lt = l + l_recv[r];
-        if (!wwait(&bar->o_done[slot], (jj >> 1) & 1)) { ok = false; break; }
+        if (!wwait(&bar->o_done[pt], (jj / kPTiles) & 1)) { ok = false; break; }
         tc_fence_after();
         const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
         const int grow_row = row0 + r;
