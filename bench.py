@@ -9,11 +9,17 @@ resident in HBM.  The default workload is DeepSeek-V3-shaped decode: 16
 sequences, 128 heads, context 32768, 64-token pages, shuffled page table.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
-device synchronise, timed with CUDA events on the launching stream; the
-latent cache (604 MB at the default workload) is larger than L2, so no L2
-flush is inserted.  Multi-GPU (torchrun): every rank runs its own replica on
-its own batch (data parallel over sequences, no collective on the data path)
-and the slowest rank's time is reported.  Rank 0 prints one JSON line.
+device synchronise, timed with two CUDA events on the launching stream and
+none in between (an event between two kernels ends the overlap of their
+launches).  When the latent cache is larger than L2 (604 MB at the default
+workload) no flush is inserted; when it fits in L2 (the V2-shaped workload)
+every step is timed alone with a 256 MB buffer rewritten before it, and the
+back-to-back (hot-L2) figure is reported beside it.  The roofline's kernel
+time is mla_decode_attn alone, timed the same way in a loop of its own after
+the steps; append, absorb and decode are also reported one by one ("phases").
+Multi-GPU (torchrun): every rank runs its own replica on its own batch (data
+parallel over sequences, no collective on the data path) and the slowest
+rank's time is reported.  Rank 0 prints one JSON line.
 
 e2e: the same K steps through the public C ABI with every step's inputs (h, q,
 positions, lengths) copied from pinned host memory and its output copied back,
@@ -55,14 +61,26 @@ METRIC = "MLA latent decode tokens/s; HBM GB/s and TFLOPS as fraction of B200 ro
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def describe(w: W.Workload) -> dict:
+L2_BYTES = 126 * 2 ** 20
+FLUSH_BYTES = 256 * 2 ** 20
+
+
+def cache_fits_l2(w: W.Workload, lens) -> bool:
+    return int(np.sum(lens)) * w.row * 2 < L2_BYTES
+
+
+def describe(w: W.Workload, lens=None) -> dict:
     d = {"workload": f"{w.name}: batch {w.batch}, {w.nq} query token(s)/seq, {w.n_heads} heads, "
                      + (f"context {w.context}" if w.context else f"context U[{w.ragged[0]},{w.ragged[1]}]")
                      + f", d_c {w.d_c}, d_rope {w.d_rope}, page {w.page_size}",
          "batch": w.batch, "nq": w.nq, "n_heads": w.n_heads, "d_c": w.d_c, "d_rope": w.d_rope,
          "qk_nope": w.qk_nope, "v_head": w.v_head, "d_model": w.d_model, "page_size": w.page_size,
-         "context": w.context if w.context else list(w.ragged), "page_table": "shuffled",
-         "l2": "inputs larger than L2: the latent cache streamed each step exceeds the 126 MB L2"}
+         "context": w.context if w.context else list(w.ragged), "page_table": "shuffled"}
+    if lens is not None and cache_fits_l2(w, lens):
+        d["l2"] = ("L2 flushed: the latent cache fits in the 126 MB L2, so a 256 MB buffer is rewritten "
+                   "before each timed step (each step timed alone)")
+    else:
+        d["l2"] = "inputs larger than L2: the latent cache streamed each step exceeds the 126 MB L2"
     return d
 
 
@@ -209,19 +227,23 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
     ws = torch.empty(M.mla_decode_workspace_bytes(dims, w.batch, w.nq), dtype=torch.uint8, device=dev)
     status = torch.zeros(4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ev_pairs = []
+    flushed = cache_fits_l2(w, x.lens)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flushed else None
 
-    def step(h_, q_, seq_idx_, pos_, seq_lens_, record=False):
+    def append_(h_, seq_idx_, pos_):
         M.mla_append_latent(dims, h_, w_dkv, seq_idx_, pos_, page_table, pool, dev_status=status, stream=stream)
+
+    def absorb_(q_, pos_):
         M.mla_absorb_q(dims, q_, pos_, w_uk, q_lat.view(T, w.n_heads, w.row), stream=stream)
-        if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+
+    def decode_(seq_lens_):
         M.mla_decode_attn(dims, q_lat, pool, page_table, seq_lens_, w_uv, ws, out, lse, dev_status=status,
                           stream=stream)
-        if record:
-            e1.record(stream)
-            ev_pairs.append((e0, e1))
+
+    def step(h_, q_, seq_idx_, pos_, seq_lens_):
+        append_(h_, seq_idx_, pos_)
+        absorb_(q_, pos_)
+        decode_(seq_lens_)
 
     launches_per_step = 4  # append, absorb, decode split, decode combine
 
@@ -231,26 +253,48 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # ---- device-resident timing
+    def timed(fn, n):
+        """Device time (ms) of n calls of fn: two events around the whole loop, or,
+        when the cache fits in L2, each call alone after an L2 flush (summed)."""
+        if not flushed:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            barrier()
+            return e0.elapsed_time(e1)
+        pairs = []
+        for _ in range(n):
+            flush_buf.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            pairs.append((e0, e1))
+        barrier()
+        return float(sum(a.elapsed_time(b) for a, b in pairs))
+
+    # ---- device-resident timing: the whole step
     for _ in range(args.warmup):
         step(h, q, seq_idx, pos, seq_lens)
     barrier()
     assert M.mla_status_read(status, stream) == 0, "device status after warm-up"
-    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    sampler = ClockSampler(local_rank)
     sampler.start()
     barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    # the decode call is timed on every 8th step: an event between two kernels
-    # ends the overlap of their launches, so timing every step would slow the loop
-    for i in range(args.steps):
-        step(h, q, seq_idx, pos, seq_lens, record=(i % 8 == 0))
-    t1.record(stream)
-    barrier()
+    ms_total = timed(lambda: step(h, q, seq_idx, pos, seq_lens), args.steps)
     clocks = sampler.stop()
-    ms_total = t0.elapsed_time(t1)
-    decode_ms = [a.elapsed_time(b) for a, b in ev_pairs]
-
+    # the same calls one by one: mla_decode_attn (the roofline's kernel time), then append and absorb
+    n_phase = min(args.steps, 200)
+    decode_ms = timed(lambda: decode_(seq_lens), n_phase) / n_phase
+    append_ms = timed(lambda: append_(h, seq_idx, pos), n_phase) / n_phase
+    absorb_ms = timed(lambda: absorb_(q, pos), n_phase) / n_phase
+    hot_ms = None
+    if flushed:   # the same steps back to back with the cache hot in L2
+        flushed = False
+        hot_ms = timed(lambda: step(h, q, seq_idx, pos, seq_lens), args.steps)
+        flushed = True
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region.
     # A serving loop's double buffering: step i's inputs go host -> device and
     # step i's output device -> host on a copy stream, overlapped with the
@@ -302,30 +346,56 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
 
     e2e_run(args.warmup)
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    last = e2e_run(args.steps, start=e0)
-    e1 = torch.cuda.Event(enable_timing=True)
-    stream.wait_event(last)
-    e1.record(stream)
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
+    if not flushed:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        last = e2e_run(args.steps, start=e0)
+        e1 = torch.cuda.Event(enable_timing=True)
+        stream.wait_event(last)
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+    else:
+        # cache in L2: each step alone after an L2 flush, its copies in and out
+        # serialised with it on one stream, timed from the first input copy to
+        # the last output copy
+        pairs = []
+        for i in range(args.steps):
+            flush_buf.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            b = dbuf[i % 2]
+            for k in host:
+                b[k].copy_(host[k], non_blocking=True)
+            M.mla_append_latent(dims, b["h"], w_dkv, b["seq_idx"], b["pos"], page_table, pool, dev_status=status,
+                                stream=stream)
+            M.mla_absorb_q(dims, b["q"], b["pos"], w_uk, q_lat.view(T, w.n_heads, w.row), stream=stream)
+            M.mla_decode_attn(dims, q_lat, pool, page_table, b["seq_lens"], w_uv, ws, outs[i % 2], lse,
+                              dev_status=status, stream=stream)
+            out_host[i % 2].copy_(outs[i % 2], non_blocking=True)
+            e1.record(stream)
+            pairs.append((e0, e1))
+        barrier()
+        e2e_ms = float(sum(a.elapsed_time(b) for a, b in pairs))
     assert M.mla_status_read(status, stream) == 0, "device status after timing"
     # the copies really happened: the last output read back equals the device result
     assert torch.equal(out_host[(args.steps - 1) % 2], outs[(args.steps - 1) % 2].cpu()), "e2e output copy"
 
-    op = measure_out_proj(M, w, dims, out, dev, stream, args.seed + rank)
-    qp = measure_query_proj(M, w, dims, dev, stream, args.seed + rank)
-    pf = measure_prefill(M, w, dims, dev, stream, args.seed + rank)
-
-    ms_total, e2e_ms, dec_ms, op_us, qp_us, pf_us = max_over_ranks(
-        [ms_total, e2e_ms, float(np.mean(decode_ms)), op["time_us"], qp["time_us"], pf["time_us"]], dev)
-    op["time_us"] = op_us
-    qp["time_us"] = qp_us
-    pf["time_us"] = pf_us
-    return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": dec_ms, "clocks": clocks,
-            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens,
-            "out_proj": op, "query_proj": qp, "prefill": pf}
+    extra = {}
+    if w.name == "v3":   # the next rows of the hot-path table, at the V3 shape
+        extra = {"out_proj": measure_out_proj(M, w, dims, out, dev, stream, args.seed + rank),
+                 "query_proj": measure_query_proj(M, w, dims, dev, stream, args.seed + rank),
+                 "prefill": measure_prefill(M, w, dims, dev, stream, args.seed + rank)}
+    keys = sorted(extra)
+    vals = max_over_ranks([ms_total, e2e_ms, decode_ms, append_ms, absorb_ms, hot_ms or 0.0]
+                          + [extra[k]["time_us"] for k in keys], dev)
+    ms_total, e2e_ms, decode_ms, append_ms, absorb_ms, hot_ms2 = vals[:6]
+    for k, v in zip(keys, vals[6:]):
+        extra[k]["time_us"] = v
+    return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": decode_ms, "decode_loop_ms": decode_ms * n_phase,
+            "phases_ms": {"append": append_ms, "absorb": absorb_ms, "decode": decode_ms},
+            "hot_ms": hot_ms2 if hot_ms is not None else None, "clocks": clocks,
+            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens, **extra}
 
 
 def measure_prefill(M, w: W.Workload, dims, dev, stream, seed: int, chunk: int = 128, batch: int = 2,
@@ -526,17 +596,21 @@ def main():
     dec_s = r["decode_ms"] / 1000.0
     gbs = cnt["bytes"] / dec_s / 1e9
     tfs = cnt["flops"] / dec_s / 1e12
+    # the decode loop runs for seconds only on the larger workloads: the tensor peak
+    # is the sustained (power-capped) figure there, the burst figure otherwise
+    tc_key = "bf16_tflops_sustained" if r["decode_loop_ms"] >= 500.0 and "bf16_tflops_sustained" in peaks \
+        else "bf16_tflops"
     t_hbm = cnt["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_tc = cnt["flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_tc = cnt["flops"] / (peaks[tc_key] * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
     roof = ({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s"} if bound == "hbm" else
-            {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"})
+            {"bound": "tensor", "achieved": tfs, "peak": peaks[tc_key], "unit": "TFLOP/s"})
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"], roof["traffic_source"] = profiled_traffic(w.name)
-    roof["kernel"] = "mla_decode_attn (split + combine launches)"
-    roof["peak_source"] = f"{src} (MEASURED_PEAKS.json burst figures)" if src == "measured" else "fallback"
+    roof["kernel"] = "mla_decode_attn (split + combine launches), timed in a loop of its own after the steps"
+    roof["peak_source"] = (f"{src} (MEASURED_PEAKS.json: hbm_gbs, {tc_key})" if src == "measured" else "fallback")
     roof["hbm_frac"] = gbs / peaks["hbm_gbs"]
-    roof["tensor_frac"] = tfs / peaks["bf16_tflops"]
+    roof["tensor_frac"] = tfs / peaks[tc_key]
     roof["time_us"] = r["decode_ms"] * 1000.0
     roof["bytes_per_launch"] = cnt["bytes"]
     roof["flops_per_launch"] = cnt["flops"]
@@ -544,33 +618,40 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r["ms_total"] / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**describe(w), "parallelism": f"dp{world} (independent replicas)"},
+            "config": {**describe(w, r["lens"]), "parallelism": f"dp{world} (independent replicas)"},
             "roofline": roof,
             "e2e": {"value": job_throughput(world, T, args.steps, r["e2e_ms"]), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                    "copies": "pinned host buffers, double-buffered on a second stream, inside the timed region"},
-            "gpu_launches": r["launches"], "clocks": r["clocks"]}
-    op = r["out_proj"]
-    op_gbs = op["bytes_per_launch"] / (op["time_us"] * 1e-6) / 1e9
-    line["next_rows"] = {"out_proj": {
-        "kernel": "token_linear_kernel (mla_out_proj), timed alone after the step, not part of it",
-        "shape": op["shape"], "bound": "hbm", "achieved": op_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-        "frac": op_gbs / peaks["hbm_gbs"], "time_us": op["time_us"], "bytes_per_launch": op["bytes_per_launch"],
-        "launches_timed": op["launches"], "l2": "W_O is larger than L2"}}
-    qp = r["query_proj"]
-    qp_gbs = qp["bytes_per_launch"] / (qp["time_us"] * 1e-6) / 1e9
-    line["next_rows"]["query_proj"] = {
-        "kernel": "token_linear_kernel x 2 (mla_query_proj), timed alone after the step, not part of it",
-        "shape": qp["shape"], "bound": "hbm", "achieved": qp_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-        "frac": qp_gbs / peaks["hbm_gbs"], "time_us": qp["time_us"], "bytes_per_call": qp["bytes_per_launch"],
-        "launches_timed": qp["launches"], "l2": "256 MB buffer rewritten before each call"}
-    pf = r["prefill"]
-    pf_tfs = pf["flops"] / (pf["time_us"] * 1e-6) / 1e12
-    line["next_rows"]["prefill"] = {
-        "kernel": "mla_decode_attn (split + combine) on a prefill chunk, timed alone after the step",
-        "shape": pf["shape"], "bound": "tensor", "achieved": pf_tfs, "peak": peaks["bf16_tflops"],
-        "unit": "TFLOP/s", "frac": pf_tfs / peaks["bf16_tflops"], "time_us": pf["time_us"],
-        "flops_per_call": pf["flops"], "launches_timed": pf["launches"]}
+                    "copies": ("pinned host buffers, double-buffered on a second stream, inside the timed region"
+                               if r["hot_ms"] is None else
+                               "pinned host buffers, each step's copies serialised with it, L2 flushed before")},
+            "gpu_launches": r["launches"], "clocks": r["clocks"],
+            "phases_us": {k: v * 1000.0 for k, v in r["phases_ms"].items()}}
+    if r["hot_ms"] is not None:
+        line["hot_l2"] = {"value": job_throughput(world, T, args.steps, r["hot_ms"]), "unit": "tokens/s",
+                          "ms_per_step": r["hot_ms"] / args.steps, "note": "the same steps back to back, cache hot in L2"}
+    if "out_proj" in r:
+        op = r["out_proj"]
+        op_gbs = op["bytes_per_launch"] / (op["time_us"] * 1e-6) / 1e9
+        line["next_rows"] = {"out_proj": {
+            "kernel": "token_linear_kernel (mla_out_proj), timed alone after the step, not part of it",
+            "shape": op["shape"], "bound": "hbm", "achieved": op_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": op_gbs / peaks["hbm_gbs"], "time_us": op["time_us"], "bytes_per_launch": op["bytes_per_launch"],
+            "launches_timed": op["launches"], "l2": "W_O is larger than L2"}}
+        qp = r["query_proj"]
+        qp_gbs = qp["bytes_per_launch"] / (qp["time_us"] * 1e-6) / 1e9
+        line["next_rows"]["query_proj"] = {
+            "kernel": "token_linear_kernel x 2 (mla_query_proj), timed alone after the step, not part of it",
+            "shape": qp["shape"], "bound": "hbm", "achieved": qp_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": qp_gbs / peaks["hbm_gbs"], "time_us": qp["time_us"], "bytes_per_call": qp["bytes_per_launch"],
+            "launches_timed": qp["launches"], "l2": "256 MB buffer rewritten before each call"}
+        pf = r["prefill"]
+        pf_tfs = pf["flops"] / (pf["time_us"] * 1e-6) / 1e12
+        line["next_rows"]["prefill"] = {
+            "kernel": "mla_decode_attn (split + combine) on a prefill chunk, timed alone after the step",
+            "shape": pf["shape"], "bound": "tensor", "achieved": pf_tfs, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": pf_tfs / peaks["bf16_tflops"], "time_us": pf["time_us"],
+            "flops_per_call": pf["flops"], "launches_timed": pf["launches"]}
     if world == 1 and not args.no_cpu_baseline:
         arm = OracleArm(w, args.seed)
         v, sample = arm.measure(args.cpu_budget)
