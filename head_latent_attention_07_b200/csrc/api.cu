@@ -80,10 +80,10 @@ struct WsLayout {
 // tensor-core path (fewer workers when there are many row tiles, as in chunked
 // prefill), else a share of two CTAs per SM over the 16-row groups.
 int decode_workers(const mla_dims* d, int nq, int sms) {
-  if (mla::decode_tc_supported(d->d_c, d->d_rope, d->page_size)) {
+  if (mla::decode_pair_supported(d->d_c, d->d_rope, d->page_size)) {
     const int tiles = (nq * d->n_heads + 127) / 128;
     const int pairs = sms / 2;
-    const int g_decode = mla::decode_tc_workers(sms, nq * d->n_heads);
+    const int g_decode = mla::decode_pair_workers(sms, nq * d->n_heads);
     if (g_decode > 1) return g_decode;   // few row tiles (decode): one wave of pairs
     // many row tiles (chunked prefill): split each tile's pages over G workers,
     // G <= 8 chosen so that the last wave of CTA pairs is as full as possible
@@ -210,9 +210,9 @@ int decode_common(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* p
   a.kv_rank = kv_rank; a.kv_ranks = kv_ranks;
   cudaStream_t s = (cudaStream_t)stream;
   a.G = decode_workers(dims, nq, sms);
-  if (mla::decode_tc_supported(dims->d_c, dims->d_rope, dims->page_size)) {
+  if (mla::decode_pair_supported(dims->d_c, dims->d_rope, dims->page_size)) {
     // tensor-core path: one CTA pair per worker and 128-row tile
-    if ((st = cuda_status(mla::launch_decode_split_tc(a, spin_limit_cycles(), s))) != MLA_OK) return st;
+    if ((st = cuda_status(mla::launch_decode_split_pair(a, spin_limit_cycles(), s))) != MLA_OK) return st;
   } else {
     if ((st = cuda_status(mla::launch_decode_split_simt(a, s))) != MLA_OK) return st;
   }

@@ -86,10 +86,11 @@ cudaError_t launch_merge_ranks(const DecodeArgs& a, const RankSources& src, cuda
 bool encode_rows576(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
                     CUtensorMapSwizzle sw);
 
-// Tensor-core split kernels (d_c = 512, d_rope = 64, 64-token pages).
-bool decode_tc_supported(int d_c, int d_rope, int page_size);
-int decode_tc_workers(int sms, int rows_total);
-cudaError_t launch_decode_split_tc(const DecodeArgs& a, long long spin_limit, cudaStream_t stream);
+// Tensor-core split kernel on CTA pairs (d_c = 512, d_rope = 64, 64-token pages).
+bool decode_pair_supported(int d_c, int d_rope, int page_size);
+// Split workers (CTA pairs) per 128-row tile when every tile gets its own set.
+int decode_pair_workers(int sms, int rows_total);
+cudaError_t launch_decode_split_pair(const DecodeArgs& a, long long spin_limit, cudaStream_t stream);
 constexpr long long kSpinLimitCycles = 1ll << 31;  // ~1 s at B200 clocks per bounded wait
 
 // Launch attribute that lets a kernel start while its predecessor on the stream

@@ -38,7 +38,7 @@ decode_split_simt_kernel(DecodeArgs a) {
   float* s_s = reinterpret_cast<float*>(page_s + a.page_size * R);                            // [kRows][P]
 
   grid_dependency_wait();
-  allow_dependent_launch();   // after the wait: see decode_tc.cu
+  allow_dependent_launch();   // only after the wait: the combine reads seq_lens and W_UV, written before this kernel's wait returned
   build_plan(&sm->plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.dev_status, a.kv_rank,
              a.kv_ranks);
   const int w = blockIdx.x;
