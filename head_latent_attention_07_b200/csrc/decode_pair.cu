@@ -22,9 +22,10 @@
 //           columns (block b holds columns 64b).  For the peer's page they held the
 //           other half of its own page, which the scores no longer need: once the
 //           step's score MMAs are done, a loader warp overwrites them with the peer
-//           page's columns [256j + 128c, +128), read from L2 with cp.async (the peer
-//           just loaded that page), and fills slots past the sequence's end with
-//           zeros.  So each CTA reads 72 KB per step from HBM and 32 KB from L2.
+//           page's columns [256j + 128c, +128), read from L2 by TMA (the peer just
+//           loaded that page); where a page is partial, per-thread copies fill slots
+//           past the sequence's end with zeros instead.  So each CTA reads 72 KB per
+//           step from HBM and 32 KB from L2.
 //
 // TMEM (512 columns, same map in both CTAs; a pair tile with M = 128 folds each
 // CTA's 64 rows into the 128 lanes: lanes [0,64) hold the first N/2 columns, lanes
@@ -38,8 +39,8 @@
 //                     lanes 64-127, j = 0 at [256,384), j = 1 at [384,512)
 //
 // Warps (256 threads per CTA): 0 loads the query and the step buffers (TMA), 1 owns
-// TMEM and, in CTA 0, issues the MMAs, 2 fetches the peer half (cp.async), 3 hands
-// the fetched half to the MMA issuer, 4-7 run the softmax and the epilogue (one
+// TMEM and, in CTA 0, issues the MMAs, 2 fetches the peer half, 3 hands a half
+// fetched by per-thread copies to the MMA issuer, 4-7 run the softmax and the epilogue (one
 // thread per TMEM lane: one row and one page).  The MMA warp runs converged: lane 0
 // tests the barriers and broadcasts its decision, one elected lane issues (an MMA
 // issued from a lone lane under data-dependent control flow costs several times
@@ -93,7 +94,7 @@ struct PairParams {
 struct Bars {
   uint64_t kfull[2];    // CTA 0: both CTAs' pages of a step landed in the step buffer (2 arrivals + bytes)
   uint64_t buf_free[2]; // both: the step's value MMAs are done with its buffer
-  uint64_t vland[2];    // local: the peer-half copies of a step have landed (32 arrivals)
+  uint64_t vland[2];    // local: per-thread peer-half copies of a partial step have landed (32 arrivals)
   uint64_t vfull[2];    // CTA 0: both CTAs' step buffers hold the value operand (2 arrivals)
   uint64_t q_full;      // CTA 0: the shared-memory part of both query halves loaded (2 arrivals + bytes)
   uint64_t qt_full;     // CTA 0: the TMEM part of the query written by the 8 softmax warps of the pair
@@ -152,6 +153,28 @@ __device__ __forceinline__ int page_id(const DecodeArgs& a, int b, int pg, int32
     return -1;
   }
   return id;
+}
+
+// What the value operand of a step needs from memory in CTA c: the peer's page
+// (id_p, or -1 when the step has no such page or it lies outside the pool) with
+// nv_p valid keys, and the number of valid keys of the own page (64 when the own
+// page is missing: its slots were zero-filled by the load).  `full` when both pages
+// are complete, so that the peer half can be copied whole by TMA; otherwise slots
+// past the sequence's end are zeroed with per-thread copies.
+struct PeerFetch {
+  int id_p, nv_p, nv_o;
+  bool full;
+};
+__device__ __forceinline__ PeerFetch peer_fetch(const DecodeArgs& a, int b, int pg0, int np, int c) {
+  PeerFetch f;
+  const int len = a.seq_lens[b];
+  const int pp = 1 - c;
+  f.id_p = pp < np ? page_id(a, b, pg0 + pp, nullptr) : -1;
+  f.nv_p = f.id_p >= 0 ? min(64, len - (pg0 + pp) * 64) : 0;
+  const int id_o = c < np ? page_id(a, b, pg0 + c, nullptr) : -1;
+  f.nv_o = id_o >= 0 ? min(64, len - (pg0 + c) * 64) : 64;
+  f.full = f.nv_p == 64 && f.nv_o == 64;
+  return f;
 }
 
 __device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
@@ -276,28 +299,43 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       ++t;
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ peer half of the value operand (cp.async)
+    // ------------------------------------------------------------ peer half of the value operand
     // Once a step's score MMAs are done, blocks 4j + 2(1-c) + e of its buffer (the
     // other half of the own page, no longer needed) receive the peer page's latent
-    // columns 256j + 128c + 64e, e = 0, 1; slots past the sequence's end are zero.
-    // The own half keeps its data, but slots of the own page past the sequence's
-    // end are zeroed too (P = 0 does not cancel NaN in the product).  Completion is
-    // signalled asynchronously on vland; warp 3 hands the step on.
+    // columns 256j + 128c + 64e, e = 0, 1, read from L2 (the peer has just loaded
+    // that page).  When both pages of the step are complete, four TMA boxes do it
+    // and count their bytes on CTA 0's vfull directly.  Otherwise per-thread copies
+    // zero the slots past the sequence's end, in the peer half and in the own half
+    // (P = 0 does not cancel NaN in the product); they signal vland, and warp 3
+    // hands the step on.
     const char* pool = reinterpret_cast<const char*>(a.pool);
+    const uint32_t vfull0 = mapa(smem_u32(&bar->vfull[0]), 0);
     StepCursor cur(plan, a.batch, w);
     Step st;
     int t = 0;
+    uint32_t n_part = 0;   // partial steps so far (they alternate between the two vland barriers)
     while (!*abort_flag && cur.next(&st)) {
       const int u = t & 1;
-      if (!wwait(&bar->s_full[u], (t >> 1) & 1)) break;
-      const int len = a.seq_lens[st.b];
       const int pp = 1 - (int)c;                                  // the peer's page of the step
-      const int id_p = pp < st.np ? page_id(a, st.b, st.pg0 + pp, nullptr) : -1;
-      const int nv_p = id_p >= 0 ? min(64, len - (st.pg0 + pp) * 64) : 0;
-      const int id_o = (int)c < st.np ? page_id(a, st.b, st.pg0 + (int)c, nullptr) : -1;
-      const int nv_o = id_o >= 0 ? min(64, len - (st.pg0 + (int)c) * 64) : 64;   // missing pages were zero-filled
-      const char* src_p = pool + (size_t)(id_p >= 0 ? id_p : 0) * 64 * 1152;
-      const uint32_t base = smem_u32(buf_s + u * kBufBytes);
+      // page ids and lengths are read before the wait, off the critical path
+      const PeerFetch f = peer_fetch(a, st.b, st.pg0, st.np, (int)c);
+      if (!wwait(&bar->s_full[u], (t >> 1) & 1)) break;
+      unsigned char* buf = buf_s + u * kBufBytes;
+      if (f.full) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx_cluster(vfull0 + 8 * u, 4 * kBlockBytes);
+          for (int je = 0; je < 4; ++je) {
+            const int j = je >> 1, e = je & 1;
+            tma_load_2d_pair(buf + (4 * j + 2 * pp + e) * kBlockBytes, &tp, 256 * j + 128 * (int)c + 64 * e,
+                             f.id_p * 64, vfull0 + 8 * u);
+          }
+        }
+        __syncwarp();
+        ++t;
+        continue;
+      }
+      const char* src_p = pool + (size_t)(f.id_p >= 0 ? f.id_p : 0) * 64 * 1152;
+      const uint32_t base = smem_u32(buf);
 #pragma unroll 1
       for (int je = 0; je < 4; ++je) {
         const int j = je >> 1, e = je & 1;
@@ -307,32 +345,37 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         for (int q = 0; q < 16; ++q) {
           const int idx = lane + 32 * q;                          // key = idx / 8, 16-byte piece = idx % 8
           const int key = idx >> 3, ch = idx & 7;
-          const bool valid = key < nv_p;
+          const bool valid = key < f.nv_p;
           cp_async16(blk_p + key * 128 + ((ch ^ (key & 7)) << 4),
                      valid ? (const void*)(src + (size_t)key * 1152 + ch * 16) : (const void*)pool, valid ? 16u : 0u);
         }
-        if (nv_o < 64) {
+        if (f.nv_o < 64) {
           const uint32_t blk_o = base + (4 * j + 2 * (int)c + e) * kBlockBytes;
-          for (int idx = nv_o * 8 + lane; idx < 512; idx += 32)
+          for (int idx = f.nv_o * 8 + lane; idx < 512; idx += 32)
             cp_async16(blk_o + (idx >> 3) * 128 + (((idx & 7) ^ ((idx >> 3) & 7)) << 4), pool, 0u);
         }
       }
-      cp_async_arrive_noinc(&bar->vland[u]);
+      cp_async_arrive_noinc(&bar->vland[n_part & 1]);
+      ++n_part;
       ++t;
     }
     cp_async_wait_all();
   } else if (warp == 3) {
-    // ------------------------------------------------------------ hand the value operand on
+    // ------------------------------------------------------------ hand a partial step's value operand on
     const uint32_t vfull0 = mapa(smem_u32(&bar->vfull[0]), 0);
     StepCursor cur(plan, a.batch, w);
     Step st;
     int t = 0;
+    uint32_t n_part = 0;
     while (cur.next(&st)) {
       const int u = t & 1;
-      if (!wwait(&bar->vland[u], (t >> 1) & 1)) break;
-      fence_proxy_async_smem();           // the copies are read by the tensor core (async proxy)
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(vfull0 + 8 * u);
+      if (!peer_fetch(a, st.b, st.pg0, st.np, (int)c).full) {
+        if (!wwait(&bar->vland[n_part & 1], (n_part >> 1) & 1)) break;
+        ++n_part;
+        fence_proxy_async_smem();           // the copies are read by the tensor core (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(vfull0 + 8 * u);
+      }
       ++t;
     }
   } else if (warp == 1) {
@@ -488,6 +531,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         const int len = a.seq_lens[st.b];
         vis = min(len - 1, len - a.nq + qi);
       }
+      // a page that the page table maps outside the pool is masked whole (its data
+      // were zero-filled); looked up before the wait, off the critical path
+      const bool pg_ok = h < st.np && page_id(a, st.b, st.pg0 + h, nullptr) >= 0;
       if (!wwait(&bar->s_full[t & 1], (t >> 1) & 1)) break;
       tc_fence_after();
       float s[64];
@@ -497,9 +543,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(s_empty0 + 8 * (t & 1));
-      // keys [0, lim_k] of page h of the step are visible to this row; a page that
-      // the page table maps outside the pool is masked whole (its data were zero-filled)
-      const bool pg_ok = h < st.np && page_id(a, st.b, st.pg0 + h, nullptr) >= 0;
+      // keys [0, lim_k] of page h of the step are visible to this row
       const int lim_k = (row_valid && pg_ok) ? min(vis - (st.pg0 + h) * 64, 63) : -1;
       float mx;
       {

@@ -36,8 +36,12 @@
  *     device unless stated.  "bf16" buffers hold IEEE bfloat16 bit patterns.
  *   - Every device pointer must be 16-byte aligned (MLA_ERR_MISALIGNED).
  *   - The caller owns every buffer.  The library allocates no device or host
- *     memory and keeps no state between calls; calls are asynchronous on
- *     `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *     memory and keeps no state between calls, with one exception:
+ *     mla_decode_attn_noalloc works in a fixed scratch array the library
+ *     defines in device memory (a static __device__ array, not an allocation)
+ *     and caches that array's address per device (see its declaration).  Calls
+ *     are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream).
  *   - Host-checkable errors return a negative mla_status before anything is
  *     launched.  Errors only the device can see (a page id outside the pool, a
  *     sequence length outside the page table, a bounded wait that ran out) are
