@@ -14,7 +14,11 @@
 //           B = the two pages at full width, CTA c supplying its own page (loaded
 //           by TMA into a step buffer: 9 blocks [64 keys x 64 columns]).  Every page
 //           crosses HBM once and each CTA receives complete 576-wide dot products.
-//   softmax per row, in the CTA that owns it (two threads per row, one per page).
+//   softmax per row, in the CTA that owns it (four threads per row: two pages times
+//           two halves of the page's keys).  P is double-buffered: block 0 (the keys
+//           of page 0) in the step buffer's rope block, which the scores no longer
+//           need, block 1 in a P block of its own per step parity; so the softmax of
+//           step t + 1 does not wait for the value MMAs of step t.
 //   values  O[128 x 512] += P[128 x 128] . C[128 x 512]  (N = 256 latent columns per
 //           MMA).  B is split by columns: for the keys of page p, CTA c supplies
 //           latent columns [256j + 128c, +128) at blocks 4j + 2p, 4j + 2p + 1 of the
@@ -38,15 +42,19 @@
 //   [256,512)         O: latent 256j + [0,128) in lanes 0-63, 256j + [128,256) in
 //                     lanes 64-127, j = 0 at [256,384), j = 1 at [384,512)
 //
-// Warps (256 threads per CTA): 0 loads the query and the step buffers (TMA), 1 owns
+// Warps (384 threads per CTA): 0 loads the query and the step buffers (TMA), 1 owns
 // TMEM and, in CTA 0, issues the MMAs, 2 fetches the peer half, 3 hands a half
-// fetched by per-thread copies to the MMA issuer, 4-7 run the softmax and the epilogue (one
-// thread per TMEM lane: one row and one page).  The MMA warp runs converged: lane 0
-// tests the barriers and broadcasts its decision, one elected lane issues (an MMA
-// issued from a lone lane under data-dependent control flow costs several times
-// its execution time).  The running max is only moved (and O rescaled in TMEM)
-// when it grows by more than 2^8.  Every mbarrier wait is bounded: on time-out the
-// kernel records MLA_ERR_TIMEOUT, stops its loops, drains its MMAs and frees TMEM.
+// fetched by per-thread copies to the MMA issuer, 4-11 run the softmax and the
+// epilogue (warps w and w + 4 share TMEM lane quarter w & 3, each reading half of
+// the columns).  The MMA warp runs converged: lane 0 tests the barriers and
+// broadcasts its decision, one elected lane issues (an MMA issued from a lone lane
+// under data-dependent control flow costs several times its execution time), and
+// it backs off when idle, leaving issue slots to the softmax warp beside it.  The
+// running max is only moved (and O rescaled in TMEM) when it grows by more than
+// 2^8.  No global load is outstanding at a release arrive on the softmax's path (a
+// release waits for it): page ids and lengths are read a step ahead.  Every
+// mbarrier wait is bounded: on time-out the kernel records MLA_ERR_TIMEOUT, stops
+// its loops, drains its MMAs and frees TMEM.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -60,17 +68,17 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kStepPages = 2;
 constexpr int kBlockBytes = 8192;             // [64 keys x 64 columns] bf16, 128-byte swizzle
 constexpr int kBufBytes = 9 * kBlockBytes;    // a step buffer: the own page at full width
 constexpr int kQBytes = 5 * kBlockBytes;      // query columns [256,576) of 64 rows
-constexpr int kPBytes = 2 * kBlockBytes;      // P [64 rows x 128 keys]
+constexpr int kPBytes = 2 * kBlockBytes;      // block 1 of P [64 rows x 128 keys] of steps t even / odd
 constexpr int kOffQ = 0;
 constexpr int kOffP = kOffQ + kQBytes;
 constexpr int kOffBuf = kOffP + kPBytes;
-constexpr int kOffXch = kOffBuf + 2 * kBufBytes;           // row maxima [2][128], row sums [128] (fp32)
-constexpr int kOffPlan = kOffXch + 3 * 128 * 4;
+constexpr int kOffXch = kOffBuf + 2 * kBufBytes;           // row maxima [2][2][128], row sums [2][128] (fp32)
+constexpr int kOffPlan = kOffXch + 6 * 128 * 4;
 constexpr int kOffBar = kOffPlan + ((int(sizeof(PlanSmem)) + 15) & ~15);
 constexpr int kNumBars = 32;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;           // TMEM base, abort flag
@@ -97,15 +105,16 @@ struct Bars {
   uint64_t vland[2];    // local: per-thread peer-half copies of a partial step have landed (32 arrivals)
   uint64_t vfull[2];    // CTA 0: both CTAs' step buffers hold the value operand (2 arrivals)
   uint64_t q_full;      // CTA 0: the shared-memory part of both query halves loaded (2 arrivals + bytes)
-  uint64_t qt_full;     // CTA 0: the TMEM part of the query written by the 8 softmax warps of the pair
+  uint64_t qt_full;     // CTA 0: the TMEM part of the query written by the 16 softmax warps of the pair
   uint64_t q_empty;     // both: the piece's score MMAs are done with the query tile
   uint64_t s_full[2];   // both: scores of a step are in TMEM (and its buffer's other half is free)
-  uint64_t s_empty[2];  // CTA 0: the 8 softmax warps of the pair have read them
-  uint64_t p_full;      // CTA 0: P of a step written (and O rescaled) in both CTAs
-  uint64_t p_empty;     // both: the value MMAs of a step are done (P free, O current)
+  uint64_t s_empty[2];  // CTA 0: the 16 softmax warps of the pair have read them
+  uint64_t p_full[2];   // CTA 0: P of a step written (and O rescaled) in both CTAs
+  uint64_t p_empty[2];  // both: the value MMAs of a step are done (O current); [t & 1] for step t, so
+                        // that a waiter (P no longer waits for them) is never two phases behind
   uint64_t o_free;      // CTA 0: the epilogue of a piece has read O in both CTAs
   uint64_t drain;       // both: every MMA issued has completed
-  uint64_t xm, xl;      // local: the 4 softmax warps published a step's row maxima / a piece's row sums
+  uint64_t xm, xl;      // local: the 8 softmax warps published a step's row maxima / a piece's row sums
 };
 static_assert(sizeof(Bars) <= kNumBars * 8, "barrier area");
 
@@ -209,8 +218,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
   unsigned char* q_s = sm + kOffQ;
   unsigned char* p_s = sm + kOffP;
   unsigned char* buf_s = sm + kOffBuf;
-  float* xch_m = reinterpret_cast<float*>(sm + kOffXch);   // [2][128]
-  float* xch_l = xch_m + 256;                              // [128]
+  float* xch_m = reinterpret_cast<float*>(sm + kOffXch);   // [step parity][key half][TMEM lane]
+  float* xch_l = xch_m + 512;                              // [key half][TMEM lane]
   PlanSmem* plan = reinterpret_cast<PlanSmem*>(sm + kOffPlan);
   Bars* bar = reinterpret_cast<Bars*>(sm + kOffBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + kOffMisc);
@@ -231,17 +240,19 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       mbar_init(&bar->vland[s], 32);
       mbar_init(&bar->vfull[s], 2);
       mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->s_empty[s], 8);
+      mbar_init(&bar->s_empty[s], 16);
     }
     mbar_init(&bar->q_full, 2);
-    mbar_init(&bar->qt_full, 8);
+    mbar_init(&bar->qt_full, 16);
     mbar_init(&bar->q_empty, 1);
-    mbar_init(&bar->p_full, 8);
-    mbar_init(&bar->p_empty, 1);
-    mbar_init(&bar->o_free, 8);
+    mbar_init(&bar->p_full[0], 16);
+    mbar_init(&bar->p_full[1], 16);
+    mbar_init(&bar->p_empty[0], 1);
+    mbar_init(&bar->p_empty[1], 1);
+    mbar_init(&bar->o_free, 16);
     mbar_init(&bar->drain, 1);
-    mbar_init(&bar->xm, 4);
-    mbar_init(&bar->xl, 4);
+    mbar_init(&bar->xm, 8);
+    mbar_init(&bar->xl, 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -407,7 +418,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
           } else {
             if (hv && tv < tq &&
                 (!sv.first || sv.p == 0 || mbar_test(&bar->o_free, (sv.p - 1) & 1)) &&
-                mbar_test(&bar->p_full, tv & 1) && mbar_test(&bar->vfull[tv & 1], (tv >> 1) & 1))
+                mbar_test(&bar->p_full[tv & 1], (tv >> 1) & 1) && mbar_test(&bar->vfull[tv & 1], (tv >> 1) & 1))
               word |= kGoV | (sv.first ? kFirstV : 0);
             if (hq && (!sq.first || (mbar_test(&bar->q_full, sq.p & 1) && mbar_test(&bar->qt_full, sq.p & 1))) &&
                 (tq < 2 || mbar_test(&bar->s_empty[tq & 1], ((tq >> 1) - 1) & 1)) &&
@@ -421,6 +432,10 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
               record_status(status, MLA_ERR_TIMEOUT);
               *abort_flag = 1;
               word = kStop;
+            } else {
+              // nothing to issue: back off, leaving the issue slots of this SM
+              // sub-partition to the softmax warp that shares it
+              __nanosleep(64);
             }
           }
         }
@@ -436,13 +451,16 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
               for (int pg = 0; pg < 2; ++pg)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {      // 16 keys of page pg per MMA
-                  const uint64_t da = smem_desc(pa + pg * kBlockBytes + ks * 32, 16, 1024, kSwizzle128);
+                  // P of page 0 sits in the step buffer's rope block, free once the
+                  // scores are done; P of page 1 in P region [tv & 1]
+                  const uint32_t pblk = pg == 0 ? bu + 8 * kBlockBytes : pa + (tv & 1) * kBlockBytes;
+                  const uint64_t da = smem_desc(pblk + ks * 32, 16, 1024, kSwizzle128);
                   const uint64_t db = smem_desc(bu + (4 * j + 2 * pg) * kBlockBytes + ks * 2048, kBlockBytes, 1024,
                                                 kSwizzle128);
                   mma_bf16_pair(tmem + kTmemO + 128 * j, da, db, id_v,
                                 ((word & kFirstV) && pg == 0 && ks == 0) ? 0u : 1u);
                 }
-            mma_commit_pair(&bar->p_empty);
+            mma_commit_pair(&bar->p_empty[tv & 1]);
             mma_commit_pair(&bar->buf_free[tv & 1]);
           }
           __syncwarp();
@@ -485,7 +503,11 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    const int quarter = warp & 3;                     // warps 4..7 -> TMEM lane quarters 0..3
+    // warps 4..11: warp w reads TMEM lane quarter w & 3 and key half kh of the
+    // step's S (columns [32 kh, 32 kh + 32)); four threads share a row: its two
+    // pages (lanes L and L ^ 64) times the two key halves
+    const int quarter = warp & 3;
+    const int kh = (warp - 4) >> 2;
     const int L = quarter * 32 + lane;                // this thread's TMEM lane
     const int r = L & 63, h = L >> 6;                 // row of this CTA, page of the step
     const int row = 64 * (int)c + r;                  // row of the tile
@@ -493,7 +515,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     const int qi = (row0 + row) / a.n_heads;          // query token of this row
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t s_empty0 = mapa(smem_u32(&bar->s_empty[0]), 0);
-    const uint32_t p_full0 = mapa(smem_u32(&bar->p_full), 0);
+    const uint32_t p_full0 = mapa(smem_u32(&bar->p_full[0]), 0);
     const uint32_t o_free0 = mapa(smem_u32(&bar->o_free), 0);
     const uint32_t qt_full0 = mapa(smem_u32(&bar->qt_full), 0);
     // latent columns [0,256) of this thread's query row into TMEM (both lanes of a
@@ -502,7 +524,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       const bool valid = row0 + row < prm.rows_total;   // rows past the tile's end read nothing
       const uint16_t* src = a.q_lat + ((size_t)s.b * prm.rows_total + row0 + row) * 576;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 2 * kh; cc < 2 * kh + 2; ++cc) {   // half of the chunks each
         uint32_t v[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -516,10 +538,17 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(qt_full0);
     };
+    // a page that the page table maps outside the pool is masked whole (its data
+    // were zero-filled); the page id and the sequence length of a step are read
+    // one step ahead, so that no load is outstanding at the arrives below (a
+    // release would wait for it)
+    auto page_ok = [&](const Step& s) { return h < s.np && page_id(a, s.b, s.pg0 + h, nullptr) >= 0; };
     StepCursor cur(plan, a.batch, w);
     Step st, nx;
     bool has = cur.next(&st);
     if (has) load_query(st);
+    bool pg_ok = has && page_ok(st);
+    int len = has ? a.seq_lens[st.b] : 0;
     float m_used = -INFINITY, l = 0.f;
     int vis = 0;    // last key index this row may see
     int t = 0;
@@ -528,57 +557,54 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       if (st.first) {
         m_used = -INFINITY;
         l = 0.f;
-        const int len = a.seq_lens[st.b];
         vis = min(len - 1, len - a.nq + qi);
       }
-      // a page that the page table maps outside the pool is masked whole (its data
-      // were zero-filled); looked up before the wait, off the critical path
-      const bool pg_ok = h < st.np && page_id(a, st.b, st.pg0 + h, nullptr) >= 0;
       if (!wwait(&bar->s_full[t & 1], (t >> 1) & 1)) break;
       tc_fence_after();
-      float s[64];
-      tmem_ld32(tmem + lane_off + 64 * (t & 1), s);
-      tmem_ld32(tmem + lane_off + 64 * (t & 1) + 32, s + 32);
+      float s[32];
+      tmem_ld32(tmem + lane_off + 64 * (t & 1) + 32 * kh, s);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(s_empty0 + 8 * (t & 1));
-      // keys [0, lim_k] of page h of the step are visible to this row
-      const int lim_k = (row_valid && pg_ok) ? min(vis - (st.pg0 + h) * 64, 63) : -1;
+      if (lane == 0) mbar_arrive_remote_relaxed(s_empty0 + 8 * (t & 1));   // the TMEM reads are complete
+      // keys [0, lim_k] of page h of the step are visible to this row, counted from
+      // this thread's first key (key 32 kh of the page)
+      const int lim_k = (row_valid && pg_ok) ? min(vis - (st.pg0 + h) * 64, 63) - 32 * kh : -1;
       float mx;
       {
-        float tt[8];
+        float tt[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) tt[i] = -INFINITY;
+        for (int i = 0; i < 4; ++i) tt[i] = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 32; ++i) {
           s[i] = i <= lim_k ? s[i] * prm.scale_log2 : -INFINITY;
-          tt[i & 7] = fmaxf(tt[i & 7], s[i]);
+          tt[i & 3] = fmaxf(tt[i & 3], s[i]);
         }
-#pragma unroll
-        for (int n = 4; n > 0; n >>= 1)
-#pragma unroll
-          for (int i = 0; i < n; ++i) tt[i] = fmaxf(tt[i], tt[i + n]);
-        mx = tt[0];
+        mx = fmaxf(fmaxf(tt[0], tt[1]), fmaxf(tt[2], tt[3]));
       }
-      // the two threads of a row (lanes L and L ^ 64, in different warps) agree on
-      // the step's row max (a bounded mbarrier, not a named barrier: a warp that
-      // gives up after a time-out must not leave the others waiting)
-      xch_m[(t & 1) * 128 + L] = mx;
+      // the four threads of a row (two pages, lanes L and L ^ 64, times two key
+      // halves) agree on the step's row max (a bounded mbarrier, not a named
+      // barrier: a warp that gives up after a time-out must not leave the others
+      // waiting)
+      float* xm_s = xch_m + (t & 1) * 256;
+      xm_s[kh * 128 + L] = mx;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->xm);
       if (!wwait(&bar->xm, t & 1)) break;
-      mx = fmaxf(mx, xch_m[(t & 1) * 128 + (L ^ 64)]);
+      mx = fmaxf(fmaxf(xm_s[L], xm_s[L ^ 64]), fmaxf(xm_s[128 + L], xm_s[128 + (L ^ 64)]));
       const float m_new = fmaxf(m_used, mx);
       const bool grow = m_new > m_used + kRescaleThreshold;
-      // the value MMAs of the previous step must be done before P is rewritten
-      // and before O is rescaled
-      if (t > 0 && !wwait(&bar->p_empty, (t - 1) & 1)) break;
+      // P is double-buffered: its blocks for this step were last read by the value
+      // MMAs of step t - 2, done before this step's buffer was loaded.  Only a
+      // rescale of O waits for the value MMAs of the previous step.  The two warps
+      // of a lane quarter hold the same rows and decide alike; each rescales its
+      // half of the row's O columns.
       if (__any_sync(0xffffffffu, grow && m_used != -INFINITY)) {
+        if (!wwait(&bar->p_empty[(t - 1) & 1], ((t - 1) >> 1) & 1)) break;
         const float alpha = (grow && m_used != -INFINITY) ? ex2(m_used - m_new) : 1.f;
         tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < 256; cc += 32) {
+        for (int cc = 128 * kh; cc < 128 * kh + 128; cc += 32) {
           float o[32];
           tmem_ld32(tmem + lane_off + kTmemO + cc, o);
           tmem_wait_ld();
@@ -592,13 +618,15 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       if (grow) m_used = m_new;
       const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
-      unsigned char* prow = p_s + h * kBlockBytes + r * 128;   // P block h: the keys of page h
+      unsigned char* prow = (h == 0 ? buf_s + (t & 1) * kBufBytes + 8 * kBlockBytes : p_s + (t & 1) * kBlockBytes) +
+                            r * 128;                   // P block h: the keys of page h
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int cq = 0; cq < 4; ++cq) {                   // 16-byte chunks 4 kh .. 4 kh + 3 of the row
+        const int ch = 4 * kh + cq;
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i = 8 * ch + 2 * e;
+          const int i = 8 * cq + 2 * e;
           const float p0 = ex2(s[i] - m_ref);                   // ex2(-inf) = 0
           const float p1 = ex2(s[i + 1] - m_ref);
           ps[e] += p0 + p1;
@@ -610,24 +638,31 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       fence_proxy_async_smem();                          // P -> tensor core (async proxy)
       tc_fence_before();                                 // O rescale -> MMA
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full0);
+      if (lane == 0) mbar_arrive_cluster(p_full0 + 8 * (t & 1));
+      // the next step's loads, issued after the release above
+      const bool pg_ok_next = has_next && page_ok(nx);
+      const int len_next = has_next ? a.seq_lens[nx.b] : 0;
 
       if (st.last) {
         // the score MMAs of this piece are done (its last S was read above): the
         // next piece's query may go into TMEM before this piece's epilogue
         if (has_next) load_query(nx);
-        // epilogue: O / l and lse of the piece; l summed over the row's two pages
-        xch_l[L] = l;
+        // epilogue: O / l and lse of the piece; l summed over the row's four
+        // threads, in the same order in each of them
+        xch_l[kh * 128 + L] = l;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->xl);
         if (!wwait(&bar->xl, st.p & 1)) break;
-        const float lt = l + xch_l[L ^ 64];
-        if (!wwait(&bar->p_empty, t & 1)) break;
+        const int l0 = L & 63;
+        const float lt = (xch_l[l0] + xch_l[128 + l0]) + (xch_l[64 + l0] + xch_l[192 + l0]);
+        // O is final once the value MMAs of this step are done (their commit also
+        // covers every earlier MMA)
+        if (!wwait(&bar->p_empty[t & 1], (t >> 1) & 1)) break;
         tc_fence_after();
         const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
         float* dst = a.part_o + ((size_t)st.id * prm.rows_total + row0 + row) * a.d_c + 128 * h;
 #pragma unroll 1
-        for (int cc = 0; cc < 256; cc += 32) {
+        for (int cc = 128 * kh; cc < 128 * kh + 128; cc += 32) {
           float o[32];
           tmem_ld32(tmem + lane_off + kTmemO + cc, o);
           tmem_wait_ld();
@@ -639,15 +674,17 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                   make_float4(o[i] * inv_l, o[i + 1] * inv_l, o[i + 2] * inv_l, o[i + 3] * inv_l);
           }
         }
-        if (row_valid && h == 0)
+        if (row_valid && h == 0 && kh == 0)
           a.part_lse[(size_t)st.id * prm.rows_total + row0 + row] =
               lt > 0.f ? (m_used + log2f(lt)) * 0.6931471805599453f : -INFINITY;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(o_free0);
+        if (lane == 0) mbar_arrive_remote_relaxed(o_free0);   // the TMEM reads are complete
       }
       st = nx;
       has = has_next;
+      pg_ok = pg_ok_next;
+      len = len_next;
       ++t;
     }
   }
