@@ -42,15 +42,13 @@
 //   [256,512)         O: latent 256j + [0,128) in lanes 0-63, 256j + [128,256) in
 //                     lanes 64-127, j = 0 at [256,384), j = 1 at [384,512)
 //
-// Warps (384 threads per CTA): 0 loads the query and the step buffers (TMA), 1 owns
-// TMEM and, in CTA 0, issues the MMAs, 2 fetches the peer half, 3 hands a half
-// fetched by per-thread copies to the MMA issuer, 4-11 run the softmax and the
-// epilogue (warps w and w + 4 share TMEM lane quarter w & 3, each reading half of
-// the columns).  The MMA warp runs converged: lane 0 tests the barriers and
-// broadcasts its decision, one elected lane issues (an MMA issued from a lone lane
-// under data-dependent control flow costs several times its execution time), and
-// it backs off when idle, leaving issue slots to the softmax warp beside it.  The
-// running max is only moved (and O rescaled in TMEM) when it grows by more than
+// Warps (416 threads per CTA): 0 loads the query and the step buffers (TMA), 1 owns
+// TMEM and, in CTA 0, issues the score MMAs, 12 (CTA 0) issues the value MMAs, 2
+// fetches the peer half, 3 hands a half fetched by per-thread copies to the value
+// issuer, 4-11 run the softmax and the epilogue (warps w and w + 4 share TMEM lane
+// quarter w & 3, each reading half of the columns).  Each MMA warp runs converged
+// and one elected lane issues (an MMA issued from a lone lane under data-dependent
+// control flow costs several times its execution time).  The running max is only moved (and O rescaled in TMEM) when it grows by more than
 // 2^8.  No global load is outstanding at a release arrive on the softmax's path (a
 // release waits for it): page ids and lengths are read a step ahead.  Every
 // mbarrier wait is bounded: on time-out the kernel records MLA_ERR_TIMEOUT, stops
@@ -68,7 +66,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 416;
 constexpr int kStepPages = 2;
 constexpr int kBlockBytes = 8192;             // [64 keys x 64 columns] bf16, 128-byte swizzle
 constexpr int kBufBytes = 9 * kBlockBytes;    // a step buffer: the own page at full width
@@ -113,7 +111,7 @@ struct Bars {
   uint64_t p_empty[2];  // both: the value MMAs of a step are done (O current); [t & 1] for step t, so
                         // that a waiter (P no longer waits for them) is never two phases behind
   uint64_t o_free;      // CTA 0: the epilogue of a piece has read O in both CTAs
-  uint64_t drain;       // both: every MMA issued has completed
+  uint64_t drain;       // both: every MMA issued has completed (a commit from each of the two issuers)
   uint64_t xm, xl;      // local: the 8 softmax warps published a step's row maxima / a piece's row sums
 };
 static_assert(sizeof(Bars) <= kNumBars * 8, "barrier area");
@@ -250,7 +248,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     mbar_init(&bar->p_empty[0], 1);
     mbar_init(&bar->p_empty[1], 1);
     mbar_init(&bar->o_free, 16);
-    mbar_init(&bar->drain, 1);
+    mbar_init(&bar->drain, 2);
     mbar_init(&bar->xm, 8);
     mbar_init(&bar->xl, 8);
     *abort_flag = 0;
@@ -390,116 +388,94 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       ++t;
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (CTA 0)
-    // Two in-order queues polled in turn: the value MMAs of step tv (first: they are
-    // on the softmax's critical path) and the score MMAs of step tq.  The whole warp
-    // runs the loop: lane 0 tests the barriers and walks the steps, the other lanes
-    // follow its decision word (broadcast by shuffle), so that the MMA operands stay
-    // warp-uniform, and one elected lane issues.
+    // ------------------------------------------------------------ score MMA issuer (CTA 0)
+    // The score and the value MMAs are issued by two warps (1 and 12), so that
+    // neither waits behind the other's issue loop (the MMA queue is shallow:
+    // issuing stalls while the tensor core works through it), and each commit
+    // tracks its own warp's MMAs only.  The whole warp runs the loop and waits;
+    // one elected lane issues (an MMA issued from a lone lane under
+    // data-dependent control flow costs several times its execution time).
     if (c == 0) {
-      constexpr uint32_t kGoV = 1, kGoK = 2, kFirstV = 4, kLastK = 8, kStop = 16;
       const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t id_v = idesc_bf16_f32(128, 256, 0, 1);
-      const uint32_t qa = smem_u32(q_s), pa = smem_u32(p_s), ba = smem_u32(buf_s);
-      StepCursor cq(plan, a.batch, w), cv(plan, a.batch, w);
-      Step sq, sv;
-      bool hq = false, hv = false;
-      int tq = 0, tv = 0;                    // steps of the two queues (all lanes)
-      if (lane == 0) {
-        hq = cq.next(&sq);
-        hv = cv.next(&sv);
-      }
-      long long t_last = clock64();
-      while (true) {
-        uint32_t word = 0;
-        if (lane == 0) {
-          if (!hq && !hv) {
-            word = kStop;
-          } else {
-            if (hv && tv < tq &&
-                (!sv.first || sv.p == 0 || mbar_test(&bar->o_free, (sv.p - 1) & 1)) &&
-                mbar_test(&bar->p_full[tv & 1], (tv >> 1) & 1) && mbar_test(&bar->vfull[tv & 1], (tv >> 1) & 1))
-              word |= kGoV | (sv.first ? kFirstV : 0);
-            if (hq && (!sq.first || (mbar_test(&bar->q_full, sq.p & 1) && mbar_test(&bar->qt_full, sq.p & 1))) &&
-                (tq < 2 || mbar_test(&bar->s_empty[tq & 1], ((tq >> 1) - 1) & 1)) &&
-                mbar_test(&bar->kfull[tq & 1], (tq >> 1) & 1))
-              word |= kGoK | (sq.last ? kLastK : 0);
-            if (word & (kGoV | kGoK)) {
-              t_last = clock64();
-            } else if (*abort_flag) {
-              word = kStop;
-            } else if (clock64() - t_last > lim) {
-              record_status(status, MLA_ERR_TIMEOUT);
-              *abort_flag = 1;
-              word = kStop;
+      const uint32_t qa = smem_u32(q_s), ba = smem_u32(buf_s);
+      StepCursor cur(plan, a.batch, w);
+      Step st;
+      int t = 0;
+      while (cur.next(&st)) {
+        if (st.first && (!wwait(&bar->q_full, st.p & 1) || !wwait(&bar->qt_full, st.p & 1))) break;
+        if (t >= 2 && !wwait(&bar->s_empty[t & 1], ((t >> 1) - 1) & 1)) break;
+        if (!wwait(&bar->kfull[t & 1], (t >> 1) & 1)) break;
+        const uint32_t bu = ba + (t & 1) * kBufBytes;
+        const uint32_t d = tmem + 64 * (t & 1);
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int ks = 0; ks < 36; ++ks) {         // 16-column steps of the 576-wide dot product
+            const uint64_t db = smem_desc(bu + (ks >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024, kSwizzle128);
+            if (ks < 16) {
+              mma_bf16_pair_ts(d, tmem + kTmemQ + 8 * ks, db, id_s, ks > 0 ? 1u : 0u);
             } else {
-              // nothing to issue: back off, leaving the issue slots of this SM
-              // sub-partition to the softmax warp that shares it
-              __nanosleep(64);
+              const uint64_t da = smem_desc(qa + ((ks - 16) >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024,
+                                            kSwizzle128);
+              mma_bf16_pair(d, da, db, id_s, 1u);
             }
           }
+          mma_commit_pair(&bar->s_full[t & 1]);
+          if (st.last) mma_commit_pair(&bar->q_empty);
         }
-        word = __shfl_sync(0xffffffffu, word, 0);
-        if (word & kStop) break;
-        if (word & kGoV) {
-          const uint32_t bu = ba + (tv & 1) * kBufBytes;
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-              for (int pg = 0; pg < 2; ++pg)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {      // 16 keys of page pg per MMA
-                  // P of page 0 sits in the step buffer's rope block, free once the
-                  // scores are done; P of page 1 in P region [tv & 1]
-                  const uint32_t pblk = pg == 0 ? bu + 8 * kBlockBytes : pa + (tv & 1) * kBlockBytes;
-                  const uint64_t da = smem_desc(pblk + ks * 32, 16, 1024, kSwizzle128);
-                  const uint64_t db = smem_desc(bu + (4 * j + 2 * pg) * kBlockBytes + ks * 2048, kBlockBytes, 1024,
-                                                kSwizzle128);
-                  mma_bf16_pair(tmem + kTmemO + 128 * j, da, db, id_v,
-                                ((word & kFirstV) && pg == 0 && ks == 0) ? 0u : 1u);
-                }
-            mma_commit_pair(&bar->p_empty[tv & 1]);
-            mma_commit_pair(&bar->buf_free[tv & 1]);
-          }
-          __syncwarp();
-          ++tv;
-          if (lane == 0) hv = cv.next(&sv);
-        }
-        if (word & kGoK) {
-          const uint32_t bu = ba + (tq & 1) * kBufBytes;
-          const uint32_t d = tmem + 64 * (tq & 1);
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int ks = 0; ks < 36; ++ks) {         // 16-column steps of the 576-wide dot product
-              const uint64_t db = smem_desc(bu + (ks >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024, kSwizzle128);
-              if (ks < 16) {
-                mma_bf16_pair_ts(d, tmem + kTmemQ + 8 * ks, db, id_s, ks > 0 ? 1u : 0u);
-              } else {
-                const uint64_t da = smem_desc(qa + ((ks - 16) >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024,
-                                              kSwizzle128);
-                mma_bf16_pair(d, da, db, id_s, 1u);
-              }
-            }
-            mma_commit_pair(&bar->s_full[tq & 1]);
-            if (word & kLastK) mma_commit_pair(&bar->q_empty);
-          }
-          __syncwarp();
-          ++tq;
-          if (lane == 0) hq = cq.next(&sq);
-        }
+        __syncwarp();
+        ++t;
       }
-      // drain: every MMA issued above has completed (and every commit before this
-      // one has arrived) before TMEM and shared memory go away
+      // drain: every MMA this warp issued has completed (and every commit before
+      // this one has arrived) before TMEM and shared memory go away; the value
+      // issuer commits to the same barrier
       if (elect_one()) mma_commit_pair(&bar->drain);
       __syncwarp();
-      if (lane == 0) mbar_wait_drain(&bar->drain, 0, kDrainCycles);
+      if (lane == 0) mbar_wait_drain(&bar->drain, 0, kDrainCycles + lim);
       __syncwarp();
     } else if (lane == 0) {
       // the leader's MMAs write this CTA's TMEM and its commits arrive here
       mbar_wait_drain(&bar->drain, 0, kDrainCycles + lim);
+    }
+  } else if (warp == 12) {
+    // ------------------------------------------------------------ value MMA issuer (CTA 0)
+    if (c == 0) {
+      const uint32_t id_v = idesc_bf16_f32(128, 256, 0, 1);
+      const uint32_t pa = smem_u32(p_s), ba = smem_u32(buf_s);
+      StepCursor cur(plan, a.batch, w);
+      Step st;
+      int t = 0;
+      while (cur.next(&st)) {
+        // the previous piece's epilogue must have read O before the first value
+        // MMA of this piece overwrites it
+        if (st.first && st.p > 0 && !wwait(&bar->o_free, (st.p - 1) & 1)) break;
+        if (!wwait(&bar->p_full[t & 1], (t >> 1) & 1)) break;
+        if (!wwait(&bar->vfull[t & 1], (t >> 1) & 1)) break;
+        const uint32_t bu = ba + (t & 1) * kBufBytes;
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int pg = 0; pg < 2; ++pg)
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {      // 16 keys of page pg per MMA
+                // P of page 0 sits in the step buffer's rope block, free once the
+                // scores are done; P of page 1 in P region [t & 1]
+                const uint32_t pblk = pg == 0 ? bu + 8 * kBlockBytes : pa + (t & 1) * kBlockBytes;
+                const uint64_t da = smem_desc(pblk + ks * 32, 16, 1024, kSwizzle128);
+                const uint64_t db = smem_desc(bu + (4 * j + 2 * pg) * kBlockBytes + ks * 2048, kBlockBytes, 1024,
+                                              kSwizzle128);
+                mma_bf16_pair(tmem + kTmemO + 128 * j, da, db, id_v, (st.first && pg == 0 && ks == 0) ? 0u : 1u);
+              }
+          mma_commit_pair(&bar->p_empty[t & 1]);
+          mma_commit_pair(&bar->buf_free[t & 1]);
+        }
+        __syncwarp();
+        ++t;
+      }
+      if (elect_one()) mma_commit_pair(&bar->drain);
+      __syncwarp();
     }
   } else {
     // ------------------------------------------------------------ softmax warps

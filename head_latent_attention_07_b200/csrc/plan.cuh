@@ -29,7 +29,8 @@ constexpr int kMinChunk = 4;      // pages: keeps per-piece overhead bounded
 
 struct PlanSmem {
   int start[kMaxBatch + 1];        // first flat page of each sequence; start[B] = total
-  int piece_begin[kMaxBatch + 1];  // first piece of each sequence; piece_begin[B] = #pieces
+  uint16_t piece_begin[kMaxBatch + 1];  // first piece of each sequence; piece_begin[B] = #pieces
+                                       // (at most workers + batch, well below 2^16)
   int chunk;                       // pages per worker
   // what the window of a sequence is computed from (see plan_win0)
   const int32_t* seq_lens;
@@ -133,10 +134,10 @@ __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens
     }
     int tot;
     int ex = block_exclusive_scan(v, ps->warp_tot, &tot);
-    if (b < batch) ps->piece_begin[b] = carry + ex;
+    if (b < batch) ps->piece_begin[b] = (uint16_t)(carry + ex);
     carry += tot;
   }
-  if (threadIdx.x == 0) ps->piece_begin[batch] = carry;
+  if (threadIdx.x == 0) ps->piece_begin[batch] = (uint16_t)carry;
   __syncthreads();
 }
 

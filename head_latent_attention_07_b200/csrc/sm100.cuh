@@ -57,12 +57,17 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the completion of the phase with the given parity.  Gives up
 // when *abort is set by another thread or after `limit` clock cycles; then it
 // records MLA_ERR_TIMEOUT (first error wins), raises *abort and returns false.
+// try_wait may suspend the thread for a while before it reports a phase still
+// open; with a budget below kPollOnlyLimit the wait polls without suspending, so
+// that a tiny budget really runs out.
+constexpr long long kPollOnlyLimit = 1ll << 16;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int32_t* dev_status, long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool poll = limit < kPollOnlyLimit;
+  if (poll ? mbar_test(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (poll ? mbar_test(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > limit) {
       record_status(dev_status, MLA_ERR_TIMEOUT);
