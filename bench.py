@@ -97,7 +97,7 @@ def algorithmic_counts(w: W.Workload, lens: np.ndarray) -> dict:
     return {"bytes": nbytes, "flops": flops, "cache_bytes": cache}
 
 
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_split_pair_v3.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_pair_kernel_v3.md")
 KERNEL_SOURCES = ["decode_pair.cu", "decode_combine.cu", "plan.cuh", "sm100.cuh", "common.cuh", "mma_frag.cuh",
                   "decode.h"]
 

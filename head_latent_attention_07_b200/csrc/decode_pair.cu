@@ -548,15 +548,18 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       const int lim_k = (row_valid && pg_ok) ? min(vis - (st.pg0 + h) * 64, 63) - 32 * kh : -1;
       float mx;
       {
+        if (lim_k < 31) {                                // keys past the visible end
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[i] = i <= lim_k ? s[i] : -INFINITY;
+        }
         float tt[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) tt[i] = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = i <= lim_k ? s[i] * prm.scale_log2 : -INFINITY;
-          tt[i & 3] = fmaxf(tt[i & 3], s[i]);
-        }
-        mx = fmaxf(fmaxf(tt[0], tt[1]), fmaxf(tt[2], tt[3]));
+        for (int i = 0; i < 32; ++i) tt[i & 3] = fmaxf(tt[i & 3], s[i]);
+        // in log2 units: the scale is positive, so the max of the scaled scores is
+        // the scaled max (rounding is monotonic); -inf stays -inf
+        mx = fmaxf(fmaxf(tt[0], tt[1]), fmaxf(tt[2], tt[3])) * prm.scale_log2;
       }
       // the four threads of a row (two pages, lanes L and L ^ 64, times two key
       // halves) agree on the step's row max (a bounded mbarrier, not a named
@@ -603,8 +606,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = 8 * cq + 2 * e;
-          const float p0 = ex2(s[i] - m_ref);                   // ex2(-inf) = 0
-          const float p1 = ex2(s[i + 1] - m_ref);
+          const float p0 = ex2(fmaf(s[i], prm.scale_log2, -m_ref));       // ex2(-inf) = 0
+          const float p1 = ex2(fmaf(s[i + 1], prm.scale_log2, -m_ref));
           ps[e] += p0 + p1;
           pk[e] = pack_bf162(p0, p1);
         }
