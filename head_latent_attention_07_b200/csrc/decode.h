@@ -72,6 +72,8 @@ struct LinearArgs {
   uint16_t* y;                // [T, N]
   int T, K, N;
   int ksplit;                 // CTAs of a cluster splitting K (1, 2, 4 or 8)
+  int w_ready;                // 1: W may be read before the dependency wait (the preceding kernel
+                              // on the stream is this call's own first launch)
 };
 
 size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);

@@ -86,13 +86,10 @@ __global__ void __launch_bounds__(kLinThreads, 4) token_linear_kernel(const Line
 #pragma unroll
   for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 
-  if (SPLIT) cluster_arrive_relaxed();  // paired with the wait before the first remote store
-  allow_dependent_launch();
-  grid_dependency_wait();  // x is written by the preceding kernel
-
   const uint4 zero = make_uint4(0, 0, 0, 0);
-  for (int s0 = s_lo + warp; s0 < s_hi; s0 += kLinWarps * U) {
-    uint4 a0[U], a1[U], b[U][NT];
+  uint4 a0[U], a1[U];
+  // the weight pieces of the batch of slices that starts at s0
+  auto load_w = [&](int s0) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int s = s0 + u * kLinWarps;
@@ -101,6 +98,24 @@ __global__ void __launch_bounds__(kLinThreads, 4) token_linear_kernel(const Line
       const bool k_ok = s < s_hi && k + 8 * q < K;
       a0[u] = (k_ok && ra_ok) ? ldg_stream(wa + k) : zero;
       a1[u] = (k_ok && rb_ok) ? ldg_stream(wb + k) : zero;
+    }
+  };
+  // W is final before the dependency wait when the preceding kernel is this call's
+  // own first launch (it lets dependents start only after its own wait): the first
+  // batch of weights is then in flight while that kernel finishes
+  if (a.w_ready) load_w(s_lo + warp);
+  if (SPLIT) cluster_arrive_relaxed();  // paired with the wait before the first remote store
+  grid_dependency_wait();  // x is written by the preceding kernel
+  allow_dependent_launch();   // after the wait: see w_ready
+  if (!a.w_ready) load_w(s_lo + warp);
+
+  for (int s0 = s_lo + warp; s0 < s_hi; s0 += kLinWarps * U) {
+    uint4 b[U][NT];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int s = s0 + u * kLinWarps;
+      const int k = 32 * s;
+      const bool k_ok = s < s_hi && k + 8 * q < K;
 #pragma unroll
       for (int j = 0; j < NT; ++j)
         b[u][j] = (k_ok && x_ok[j]) ? __ldg(reinterpret_cast<const uint4*>(xr[j] + k)) : zero;
@@ -109,6 +124,7 @@ __global__ void __launch_bounds__(kLinThreads, 4) token_linear_kernel(const Line
     for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int j = 0; j < NT; ++j) mma_k32(acc[j], a0[u], a1[u], b[u][j]);
+    if (s0 + kLinWarps * U < s_hi) load_w(s0 + kLinWarps * U);
   }
 
 #pragma unroll
@@ -179,12 +195,20 @@ cudaError_t launch_nt(const LinearArgs& a, cudaStream_t stream) {
 }  // namespace
 
 int linear_ksplit(int N, int K, int sms) {
-  // enough CTAs for two per SM when W has few rows, while each split CTA keeps
-  // at least 16 slices (512 columns) of every row
+  // The split (cluster size, 1..8) whose CTAs fill their last wave best (four CTAs
+  // per SM are resident), while each split CTA keeps at least 16 slices (512
+  // columns) of every row; ties go to the smaller split.
   const int tiles = (N + kLinRows - 1) / kLinRows;
-  int ks = 1;
-  while (ks < kLinMaxSplit && tiles * ks < 2 * sms && (K / 32) / (2 * ks) >= 16) ks *= 2;
-  return ks;
+  const int slots = 4 * sms;
+  int best = 1;
+  double best_fill = 0.0;
+  for (int ks = 1; ks <= kLinMaxSplit; ++ks) {
+    if (ks > 1 && (K / 32) / ks < 16) break;
+    const long long ctas = (long long)tiles * ks;
+    const double fill = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
+    if (fill > best_fill + 0.02) { best_fill = fill; best = ks; }
+  }
+  return best;
 }
 
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t stream) {
