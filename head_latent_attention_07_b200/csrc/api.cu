@@ -210,7 +210,9 @@ int decode_common(const mla_dims* dims, const mla_bf16* q_lat, const mla_bf16* p
   a.kv_rank = kv_rank; a.kv_ranks = kv_ranks;
   cudaStream_t s = (cudaStream_t)stream;
   a.G = decode_workers(dims, nq, sms);
-  if (mla::decode_pair_supported(dims->d_c, dims->d_rope, dims->page_size)) {
+  const bool pair = mla::decode_pair_supported(dims->d_c, dims->d_rope, dims->page_size);
+  a.piece_cost = pair ? mla::kPairPieceCost : 0;
+  if (pair) {
     // tensor-core path: one CTA pair per worker and 128-row tile
     if ((st = cuda_status(mla::launch_decode_split_pair(a, spin_limit_cycles(), s))) != MLA_OK) return st;
   } else {
@@ -282,7 +284,6 @@ int mla_out_proj(const mla_dims* dims, const mla_bf16* o, const mla_bf16* w_o, m
   a.x = o; a.w = w_o; a.y = y;
   a.T = n_tokens; a.K = dims->n_heads * dims->v_head; a.N = dims->d_model;
   a.ksplit = mla::linear_ksplit(a.N, a.K, sms);
-  a.w_ready = 0;
   return cuda_status(mla::launch_linear(a, (cudaStream_t)stream));
 }
 
@@ -303,13 +304,11 @@ int mla_query_proj(const mla_dims* dims, int32_t q_lora_rank, const mla_bf16* h,
   down.x = h; down.w = w_dq; down.y = c_q;
   down.T = n_tokens; down.K = dims->d_model; down.N = q_lora_rank;
   down.ksplit = mla::linear_ksplit(down.N, down.K, sms);
-  down.w_ready = 0;
   if ((st = cuda_status(mla::launch_linear(down, s))) != MLA_OK) return st;
   mla::LinearArgs up;                          // [q_nope || q_rope] per head = W_UQ c_Q
   up.x = c_q; up.w = w_uq; up.y = q;
   up.T = n_tokens; up.K = q_lora_rank; up.N = dims->n_heads * (dims->qk_nope + dims->d_rope);
   up.ksplit = mla::linear_ksplit(up.N, up.K, sms);
-  up.w_ready = 1;   // the preceding kernel is `down`, which lets this one start only after its own wait
   return cuda_status(mla::launch_linear(up, s));
 }
 

@@ -31,8 +31,6 @@ append_latent_kernel(AppendArgs a) {
   // split cluster barrier: the wait before the first remote store below makes sure
   // every CTA of the cluster (the leader included) has started
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-  allow_dependent_launch();
-  grid_dependency_wait();
   const int R = a.d_c + a.d_rope;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, q = lane & 3;
@@ -45,9 +43,10 @@ append_latent_kernel(AppendArgs a) {
   const uint4 z = make_uint4(0, 0, 0, 0);
   float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
   const int nslices = (a.d_model + 31) / 32;
-  // slices of this CTA's quarter, interleaved over its warps; 4 per batch of loads
-  for (int base = split * kAppWarps + warp; base < nslices; base += 4 * kAppWarps * kAppSplit) {
-    uint4 ra[4], rb[4], ha[4], hb[4];
+  // slices of this CTA's eighth, interleaved over its warps; 4 per batch of loads
+  constexpr int kStride = 4 * kAppWarps * kAppSplit;
+  uint4 ra[4], rb[4];
+  auto load_w = [&](int base) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int sl = base + u * kAppWarps * kAppSplit;
@@ -55,6 +54,22 @@ append_latent_kernel(AppendArgs a) {
       const bool kin = sl < nslices && kk < a.d_model;
       ra[u] = (kin && ra_row < R) ? ldg_stream(a.w_dkv + (size_t)ra_row * a.d_model + kk) : z;
       rb[u] = (kin && rb_row < R) ? ldg_stream(a.w_dkv + (size_t)rb_row * a.d_model + kk) : z;
+    }
+  };
+  // The weights are read before the dependency wait, while the preceding kernel
+  // on the stream finishes (no kernel of this library writes weights; the header
+  // states the caller's side: the kernel enqueued just before the call must not
+  // write them).
+  load_w(split * kAppWarps + warp);
+  grid_dependency_wait();   // h, the page table and the pool may be written by the preceding kernel
+  allow_dependent_launch();
+  for (int base = split * kAppWarps + warp; base < nslices; base += kStride) {
+    uint4 ha[4], hb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sl = base + u * kAppWarps * kAppSplit;
+      const int kk = sl * 32 + 8 * q;
+      const bool kin = sl < nslices && kk < a.d_model;
       ha[u] = (kin && ta < a.n_tokens) ? *reinterpret_cast<const uint4*>(a.h + (size_t)ta * a.d_model + kk) : z;
       hb[u] = (kin && tb < a.n_tokens) ? *reinterpret_cast<const uint4*>(a.h + (size_t)tb * a.d_model + kk) : z;
     }
@@ -63,6 +78,7 @@ append_latent_kernel(AppendArgs a) {
       mma_k32(d0, ra[u], rb[u], ha[u]);
       mma_k32(d1, ra[u], rb[u], hb[u]);
     }
+    if (base + kStride < nslices) load_w(base + kStride);
   }
   // fragment -> part[warp][row][token]
 #pragma unroll
@@ -155,8 +171,6 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
 __global__ void __launch_bounds__(kAbsThreads)
 absorb_q_mma_kernel(AbsorbArgs a) {
   extern __shared__ __align__(16) uint16_t wsm[];   // [qk_nope][d_c + 8]
-  allow_dependent_launch();
-  grid_dependency_wait();
   const int h = blockIdx.x;
   const int t0 = blockIdx.y * kTokBlk;
   const int dq = a.qk_nope + a.d_rope;
@@ -174,6 +188,10 @@ absorb_q_mma_kernel(AbsorbArgs a) {
                  : "memory");
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
+  // W_UK,h streams in before the dependency wait, while the preceding kernel on
+  // the stream finishes (as in the append kernel above).
+  grid_dependency_wait();   // q may be written by the preceding kernel
+  allow_dependent_launch();
   // A fragments (q_nope of this warp's 16 tokens) for every k step, loaded once
   // while W_UK,h streams in
   const int ta = t0 + g, tb = t0 + g + 8;
@@ -226,8 +244,8 @@ absorb_q_mma_kernel(AbsorbArgs a) {
 __global__ void __launch_bounds__(kAbsThreads)
 absorb_q_kernel(AbsorbArgs a) {
   extern __shared__ __align__(16) float qn[];   // [kTokBlk][qk_nope]
-  allow_dependent_launch();
   grid_dependency_wait();
+  allow_dependent_launch();
   const int h = blockIdx.x;
   const int t0 = blockIdx.y * kTokBlk;
   const int dq = a.qk_nope + a.d_rope;

@@ -15,6 +15,12 @@ inline void rope_inv_freq(double* out, int d_rope, float theta) {
   for (int i = 0; i < d_rope / 2 && i < kMaxRopePairs; ++i) out[i] = pow((double)theta, -2.0 * i / d_rope);
 }
 
+// Per-piece overhead of the tensor-core split kernel, in pages of work: loading
+// the next piece's query, writing a partial and refilling the pipeline.  A clock
+// trace at the v3 workload showed the workers whose chunk crossed a sequence
+// start finishing ~6 % (about 7 pages of 111) after the others.
+constexpr int kPairPieceCost = 8;
+
 struct DecodeArgs {
   const uint16_t* q_lat;      // [B, nq, H, R]
   const uint16_t* pool;       // [num_pages, P, R]
@@ -30,6 +36,7 @@ struct DecodeArgs {
                               // output (and lse) instead of applying W_UV (context split)
   int batch, nq, n_heads, d_c, d_rope, v_head, page_size, max_pages, num_pages;
   int G;                      // split workers
+  int piece_cost;             // per-piece overhead of the split kernel, in pages (plan.cuh)
   int kv_rank, kv_ranks;      // context split: this call takes window kv_rank of kv_ranks
   float scale;
 };
@@ -72,8 +79,6 @@ struct LinearArgs {
   uint16_t* y;                // [T, N]
   int T, K, N;
   int ksplit;                 // CTAs of a cluster splitting K (1, 2, 4 or 8)
-  int w_ready;                // 1: W may be read before the dependency wait (the preceding kernel
-                              // on the stream is this call's own first launch)
 };
 
 size_t decode_simt_smem_bytes(int d_c, int d_rope, int page_size);

@@ -94,20 +94,22 @@ decode_combine_kernel(DecodeArgs a, const __grid_constant__ RankSources src, int
   };
 
   const bool lat_mode = !RANKS && a.out_lat != nullptr;
-  allow_dependent_launch();
   if (RANKS) {
-    // the predecessor is the caller's: wait before reading anything
-    grid_dependency_wait();
+    // the predecessor is the caller's: only the weight slice is read before the
+    // wait (the kernel enqueued just before the call must not write W_UV)
     stage_w(0);
+    grid_dependency_wait();
   } else {
     // The predecessor on the stream is always this call's split kernel, which
     // writes only the partials and lets this kernel launch only after its own
     // dependency wait: seq_lens and W_UV are final here, the partials after the
     // wait below.
     if (!lat_mode) stage_w(0);
-    build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, nullptr, a.kv_rank, a.kv_ranks);
+    build_plan(ps, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.piece_cost, nullptr, a.kv_rank,
+               a.kv_ranks);
     grid_dependency_wait();   // the split kernel's partials
   }
+  allow_dependent_launch();   // after the wait, as in every kernel here
 
   // 1. merge: 16 threads per token, each owning columns [8 gc, 8 gc + 8) and
   //    [128 + 8 gc, 128 + 8 gc + 8) of the slice; one pass over the pieces in

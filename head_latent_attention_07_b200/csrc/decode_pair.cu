@@ -267,7 +267,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
   // only now may the combine launch: its prologue reads seq_lens and W_UV,
   // whose producers (if any) ran before this kernel's wait returned
   allow_dependent_launch();
-  build_plan(plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G,
+  build_plan(plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.piece_cost,
              (blockIdx.x == 0 && blockIdx.y == 0) ? status : nullptr, a.kv_rank, a.kv_ranks);  // ends with __syncthreads
   tc_fence_before();
   cluster_sync();  // barriers and TMEM of both CTAs ready before any remote traffic

@@ -39,15 +39,10 @@ decode_split_simt_kernel(DecodeArgs a) {
 
   grid_dependency_wait();
   allow_dependent_launch();   // only after the wait: the combine reads seq_lens and W_UV, written before this kernel's wait returned
-  build_plan(&sm->plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.dev_status, a.kv_rank,
-             a.kv_ranks);
+  build_plan(&sm->plan, a.seq_lens, a.batch, a.nq, a.max_pages, a.page_size, a.G, a.piece_cost, a.dev_status,
+             a.kv_rank, a.kv_ranks);
   const int w = blockIdx.x;
   const int row0 = blockIdx.y * kRows;
-  const int chunk = sm->plan.chunk;
-  const int total = sm->plan.start[a.batch];
-  const int f0 = w * chunk;
-  const int f1 = min(f0 + chunk, total);
-  if (f0 >= f1) return;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int P = a.page_size;
@@ -58,13 +53,11 @@ decode_split_simt_kernel(DecodeArgs a) {
   const int rq = (tid / 64) * 4;
   const bool own_cols = cv < a.d_c / 8;
 
-  int b = seq_of_flat_page(&sm->plan, a.batch, f0);
-  int f = f0;
-  while (f < f1) {
-    while (sm->plan.start[b + 1] <= f) ++b;  // skip empty sequences
-    const int sb = sm->plan.start[b];
-    const int seg_end = min(f1, sm->plan.start[b + 1]);
-    const int piece = sm->plan.piece_begin[b] + (w - sb / chunk);
+  PieceIter it(&sm->plan, a.batch, w);
+  Piece pc;
+  while (it.next(&pc)) {
+    const int b = pc.b;
+    const int piece = pc.id;
     const int len = a.seq_lens[b];
 
     // query rows of this sequence -> fp32 shared memory
@@ -90,8 +83,7 @@ decode_split_simt_kernel(DecodeArgs a) {
       for (int k = 0; k < 8; ++k) acc[r][k] = 0.f;
     __syncthreads();
 
-    const int w0 = plan_win0(&sm->plan, b);   // pages are indexed from the sequence's start
-    for (int pg = f - sb + w0; pg < seg_end - sb + w0; ++pg) {
+    for (int pg = pc.pg_begin; pg < pc.pg_end; ++pg) {   // absolute page indices of the sequence
       const int page_id = a.page_table[(size_t)b * a.max_pages + pg];
       if (page_id < 0 || page_id >= a.num_pages) {  // uniform across the CTA
         if (tid == 0) record_status(a.dev_status, MLA_ERR_RANGE);
@@ -204,7 +196,6 @@ decode_split_simt_kernel(DecodeArgs a) {
       pl[row0 + tid] = l > 0.f ? (sm->m[tid] + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
-    f = seg_end;
   }
 }
 

@@ -100,14 +100,14 @@ __global__ void __launch_bounds__(kLinThreads, 4) token_linear_kernel(const Line
       a1[u] = (k_ok && rb_ok) ? ldg_stream(wb + k) : zero;
     }
   };
-  // W is final before the dependency wait when the preceding kernel is this call's
-  // own first launch (it lets dependents start only after its own wait): the first
-  // batch of weights is then in flight while that kernel finishes
-  if (a.w_ready) load_w(s_lo + warp);
+  // The first batch of weights is in flight before the dependency wait, while the
+  // preceding kernel on the stream finishes (the kernel enqueued just before the
+  // call must not write W; every kernel here allows its dependents only after its
+  // own wait, so everything earlier on the stream has completed).
+  load_w(s_lo + warp);
   if (SPLIT) cluster_arrive_relaxed();  // paired with the wait before the first remote store
   grid_dependency_wait();  // x is written by the preceding kernel
-  allow_dependent_launch();   // after the wait: see w_ready
-  if (!a.w_ready) load_w(s_lo + warp);
+  allow_dependent_launch();
 
   for (int s0 = s_lo + warp; s0 < s_hi; s0 += kLinWarps * U) {
     uint4 b[U][NT];
@@ -195,20 +195,12 @@ cudaError_t launch_nt(const LinearArgs& a, cudaStream_t stream) {
 }  // namespace
 
 int linear_ksplit(int N, int K, int sms) {
-  // The split (cluster size, 1..8) whose CTAs fill their last wave best (four CTAs
-  // per SM are resident), while each split CTA keeps at least 16 slices (512
-  // columns) of every row; ties go to the smaller split.
+  // enough CTAs for two per SM when W has few rows, while each split CTA keeps
+  // at least 16 slices (512 columns) of every row
   const int tiles = (N + kLinRows - 1) / kLinRows;
-  const int slots = 4 * sms;
-  int best = 1;
-  double best_fill = 0.0;
-  for (int ks = 1; ks <= kLinMaxSplit; ++ks) {
-    if (ks > 1 && (K / 32) / ks < 16) break;
-    const long long ctas = (long long)tiles * ks;
-    const double fill = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
-    if (fill > best_fill + 0.02) { best_fill = fill; best = ks; }
-  }
-  return best;
+  int ks = 1;
+  while (ks < kLinMaxSplit && tiles * ks < 2 * sms && (K / 32) / (2 * ks) >= 16) ks *= 2;
+  return ks;
 }
 
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t stream) {

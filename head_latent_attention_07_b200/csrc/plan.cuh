@@ -1,15 +1,19 @@
 // Split-KV schedule shared by the decode split kernels and the combine kernel.
 //
-// The pages of all sequences are laid end to end (sequence 0's pages, then
-// sequence 1's, ...).  That flat list is cut into contiguous chunks of `chunk`
-// pages; worker w processes flat pages [w*chunk, (w+1)*chunk).  A worker's chunk
-// may end inside one sequence and continue into the next.  Each overlap of a
-// worker with a sequence is a "piece"; a piece writes one partial result
-// (softmax-normalised latent output and log-sum-exp per row) to the workspace.
-// The pieces of sequence b are consecutive: piece_begin[b] .. piece_begin[b] +
-// npieces[b] - 1, worker w's piece of b being piece_begin[b] + (w - w_first[b]).
-// With chunk >= ceil(total / G) at most G workers are busy, so there are at
-// most G + batch - 1 pieces.
+// The pages of all sequences are laid end to end on a cost axis (sequence 0's
+// pages, then sequence 1's, ...), each non-empty sequence preceded by
+// `piece_cost` units that hold no page: the time a worker spends starting and
+// finishing a piece (query load, partial write, pipeline refill), in pages.
+// That axis is cut into contiguous chunks of `chunk` units; worker w takes the
+// pages at positions [w*chunk, (w+1)*chunk).  A worker's chunk may end inside
+// one sequence and continue into the next, and a worker whose chunk crosses a
+// sequence start is given correspondingly fewer pages.  Each overlap of a
+// worker with a sequence's pages is a "piece"; a piece writes one partial
+// result (softmax-normalised latent output and log-sum-exp per row) to the
+// workspace.  The pieces of sequence b are consecutive: piece_begin[b] ..
+// piece_begin[b] + npieces[b] - 1, worker w's piece of b being piece_begin[b] +
+// (w - w_first[b]).  With chunk >= ceil(total / G) at most G workers are busy,
+// so there are at most G + batch - 1 pieces.
 //
 // Every CTA rebuilds this schedule from seq_lens in shared memory (two block
 // scans over the batch), so no planning launch and no metadata buffer exist.
@@ -28,10 +32,11 @@ constexpr int kMaxBatch = 1024;   // sequences per decode call
 constexpr int kMinChunk = 4;      // pages: keeps per-piece overhead bounded
 
 struct PlanSmem {
-  int start[kMaxBatch + 1];        // first flat page of each sequence; start[B] = total
+  int start[kMaxBatch + 1];        // cost-axis position of each sequence's first page; start[B] = total
+  int npg[kMaxBatch];              // pages of each sequence (in this rank's window)
   uint16_t piece_begin[kMaxBatch + 1];  // first piece of each sequence; piece_begin[B] = #pieces
                                        // (at most workers + batch, well below 2^16)
-  int chunk;                       // pages per worker
+  int chunk;                       // cost units per worker
   // what the window of a sequence is computed from (see plan_win0)
   const int32_t* seq_lens;
   int nq, max_pages, page_size, kv_rank, kv_ranks;
@@ -93,11 +98,12 @@ __device__ __forceinline__ int plan_win0(const PlanSmem* ps, int b) {
   return window_begin(pages, ps->kv_rank, ps->kv_ranks);
 }
 
-// Fills ps->start, ps->piece_begin, ps->chunk and the window parameters for `batch` sequences
-// and G workers, over the windows of rank kv_rank of kv_ranks.
+// Fills ps->start, ps->npg, ps->piece_begin, ps->chunk and the window parameters for
+// `batch` sequences and G workers, over the windows of rank kv_rank of kv_ranks.
 __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens, int batch, int nq, int max_pages,
-                           int page_size, int G, int32_t* dev_status, int kv_rank = 0, int kv_ranks = 1) {
-  // pass 1: pages per sequence (in this rank's window) -> start offsets
+                           int page_size, int G, int piece_cost, int32_t* dev_status, int kv_rank = 0,
+                           int kv_ranks = 1) {
+  // pass 1: pages per sequence (in this rank's window) -> cost-axis positions
   int carry = 0;
   for (int base = 0; base < batch; base += blockDim.x) {
     int b = base + threadIdx.x;
@@ -105,9 +111,13 @@ __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens
                                   blockIdx.x == 0 && blockIdx.y == 0 ? dev_status : nullptr)
                       : 0;
     if (b < batch) v = window_begin(v, kv_rank + 1, kv_ranks) - window_begin(v, kv_rank, kv_ranks);
+    const int lead = v > 0 ? piece_cost : 0;
     int tot;
-    int ex = block_exclusive_scan(v, ps->warp_tot, &tot);
-    if (b < batch) ps->start[b] = carry + ex;
+    int ex = block_exclusive_scan(v + lead, ps->warp_tot, &tot);
+    if (b < batch) {
+      ps->start[b] = carry + ex + lead;
+      ps->npg[b] = v;
+    }
     carry += tot;
   }
   if (threadIdx.x == 0) {
@@ -129,8 +139,8 @@ __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens
     int b = base + threadIdx.x;
     int v = 0;
     if (b < batch) {
-      int s = ps->start[b], e = ps->start[b + 1];
-      v = e > s ? (e - 1) / chunk - s / chunk + 1 : 0;
+      const int s = ps->start[b], n = ps->npg[b];
+      v = n > 0 ? (s + n - 1) / chunk - s / chunk + 1 : 0;
     }
     int tot;
     int ex = block_exclusive_scan(v, ps->warp_tot, &tot);
@@ -141,14 +151,15 @@ __device__ __forceinline__ void build_plan(PlanSmem* ps, const int32_t* seq_lens
   __syncthreads();
 }
 
-// Sequence containing flat page f (start[b] <= f < start[b+1]); f < total.
-__device__ __forceinline__ int seq_of_flat_page(const PlanSmem* ps, int batch, int f) {
+// The last sequence whose first page lies at or before cost position f (0 if
+// none); f < total.  Its pages may end before f: the iterator skips ahead.
+__device__ __forceinline__ int seq_at_position(const PlanSmem* ps, int batch, int f) {
   int lo = 0, hi = batch - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
     if (ps->start[mid] <= f) lo = mid; else hi = mid - 1;
   }
-  return lo;  // the largest such b, so empty sequences sharing its start are skipped
+  return lo;
 }
 
 // One (sequence, page range) overlap of this worker's chunk.
@@ -165,16 +176,19 @@ struct PieceIter {
     const int total = ps->start[batch];
     f = w * chunk;
     f1 = min(f + chunk, total);
-    b = f < f1 ? seq_of_flat_page(ps, batch, f) : 0;
+    b = f < f1 ? seq_at_position(ps, batch, f) : 0;
   }
   __device__ bool next(Piece* p) {
-    if (f >= f1) return false;
-    while (ps->start[b + 1] <= f) ++b;
+    // skip empty sequences and those whose pages end before f
+    while (b < batch && (ps->npg[b] == 0 || ps->start[b] + ps->npg[b] <= f)) ++b;
+    if (b >= batch) return false;
     const int sb = ps->start[b];
-    const int e = min(f1, ps->start[b + 1]);
+    const int s = max(f, sb);
+    if (s >= f1) return false;
+    const int e = min(f1, sb + ps->npg[b]);
     const int w0 = plan_win0(ps, b);
     p->b = b;
-    p->pg_begin = f - sb + w0;   // absolute page indices of the sequence
+    p->pg_begin = s - sb + w0;   // absolute page indices of the sequence
     p->pg_end = e - sb + w0;
     p->id = ps->piece_begin[b] + (w - sb / chunk);
     f = e;

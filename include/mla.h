@@ -51,6 +51,13 @@
  *     after about 2^31 cycles (~1 s), records MLA_ERR_TIMEOUT and ends the kernel
  *     cleanly.  The environment variable MLA_SPIN_LIMIT (cycles, read at each
  *     call) overrides the budget; tests set it small to exercise that path.
+ *   - Overlap with the preceding kernel: every kernel is launched with
+ *     programmatic dependent launch and may start while the kernel enqueued
+ *     just before it on `stream` finishes.  Activations, caches, page tables
+ *     and lengths are read only after waiting for that kernel; weight matrices
+ *     (w_dkv, w_uk, w_uv, w_o, w_dq, w_uq) may be read before, so the kernel
+ *     enqueued immediately before a call must not write a weight that the call
+ *     reads (any earlier work on the stream may).
  *   - RoPE: channel pair (2i, 2i+1) rotates by pos * theta^(-2i/d_rope), the
  *     angle evaluated in double precision; pos = cache index of the token.
  *   - bf16 outputs are rounded to nearest even from fp32 accumulators.
