@@ -37,6 +37,11 @@ tensor peak.
 
 --impl reference times the CPU oracle (float64 numpy, absorbed form) on a
 bounded sample of the same workload on the host cores, as the comparison arm.
+
+--prefill-forms prints one JSON line comparing, on chunks of 128 to 1024 new
+tokens per sequence (2 sequences of 32768, V3 heads), this library's absorbed
+prefill with the decompressing form built from library kernels (cuBLAS GEMMs
+and fused attention through torch), to place their crossover.
 """
 from __future__ import annotations
 
@@ -432,6 +437,92 @@ def measure_prefill(M, w: W.Workload, dims, dev, stream, seed: int, chunk: int =
             "shape": f"{batch} sequences x {chunk} new tokens, context {context}, {wp.n_heads} heads"}
 
 
+def measure_prefill_naive(w: W.Workload, dev, stream, seed: int, chunk: int, batch: int = 2,
+                          context: int = 32768, iters: int = 3) -> dict:
+    """The decompressing (naive) form of the same prefill chunk, for comparison with
+    the absorbed form this library implements: K_nope = c W_UK^T and V = c W_UV^T for
+    every cached token and head (cuBLAS bf16 GEMMs through torch), then attention of
+    the chunk's queries over [K_nope || k_R] and V with torch's fused attention
+    (cuDNN, else the memory-efficient kernel).  Library kernels, timed only to place
+    the crossover; the gather of the paged cache into contiguous rows is not timed,
+    and the causal mask inside the chunk is left out (it covers chunk^2 / 2 of the
+    chunk x context scores)."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    wp = dataclasses.replace(w, name="prefill", batch=batch, nq=chunk, context=context)
+    x = W.make_decode_inputs(wp, seed=seed)
+    to_bf16 = lambda b: torch.from_numpy(np.ascontiguousarray(b)).view(torch.bfloat16).to(dev)
+    pool = to_bf16(x.bits["pool"])
+    pt = torch.from_numpy(np.ascontiguousarray(x.page_table, dtype=np.int64)).to(dev)
+    H, dn, dr, dv, dc = wp.n_heads, wp.qk_nope, wp.d_rope, wp.v_head, wp.d_c
+    rows = pool[pt].reshape(batch, -1, wp.row)[:, :context]          # [B, N, d_c + d_rope], untimed gather
+    c = rows[..., :dc].reshape(-1, dc).contiguous()
+    k_r = rows[..., dc:].contiguous()
+    w_uk = to_bf16(x.bits["w_uk"]).reshape(H * dn, dc)             # [H, d_h, d_c] rows
+    w_uv = to_bf16(x.bits["w_uv"]).reshape(H * dv, dc)             # [H, d_v, d_c] rows
+    q = to_bf16(x.bits["q"]).reshape(batch, chunk, H, dn + dr).transpose(1, 2)
+    N = context
+
+    def decompress():
+        k_n = (c @ w_uk.t()).view(batch, N, H, dn)
+        v = (c @ w_uv.t()).view(batch, N, H, dv)
+        k = torch.cat([k_n, k_r.view(batch, N, 1, dr).expand(batch, N, H, dr)], dim=-1)
+        return k.transpose(1, 2), v.transpose(1, 2)
+
+    backend = None
+    for b in (SDPBackend.CUDNN_ATTENTION, SDPBackend.EFFICIENT_ATTENTION):
+        try:
+            with sdpa_kernel([b]):
+                k, v = decompress()
+                F.scaled_dot_product_attention(q, k, v)
+            backend = b
+            break
+        except RuntimeError:
+            continue
+    if backend is None:
+        return {"chunk": chunk, "unavailable": "no fused attention backend takes d_qk 192, d_v 128 here"}
+    torch.cuda.synchronize(dev)
+    t_dec, t_att = [], []
+    with torch.cuda.stream(stream), sdpa_kernel([backend]):
+        for _ in range(iters + 1):
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            k, v = decompress()
+            e1.record(stream)
+            F.scaled_dot_product_attention(q, k, v)
+            e2.record(stream)
+            t_dec.append((e0, e1))
+            t_att.append((e1, e2))
+            del k, v
+    torch.cuda.synchronize(dev)
+    dec = float(np.mean([a.elapsed_time(b) for a, b in t_dec[1:]])) * 1000.0
+    att = float(np.mean([a.elapsed_time(b) for a, b in t_att[1:]])) * 1000.0
+    flops = batch * (2 * N * dc * H * (dn + dv) + 2 * chunk * N * H * (dn + dr + dv))
+    return {"chunk": chunk, "time_us": dec + att, "decompress_us": dec, "attention_us": att, "flops": flops,
+            "attention_backend": str(backend).split(".")[-1]}
+
+
+def prefill_forms(args, w: W.Workload) -> None:
+    """One JSON line: the absorbed form (this library's mla_decode_attn) against the
+    decompressing form (library kernels) on prefill chunks of V3 heads over 32K keys."""
+    import torch
+    import head_latent_attention_07_b200 as M
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    dims = M.MlaDims(n_heads=w.n_heads, d_c=w.d_c, d_rope=w.d_rope, qk_nope=w.qk_nope, v_head=w.v_head,
+                     d_model=w.d_model, page_size=w.page_size)
+    rows = []
+    for chunk in (128, 256, 512, 1024):
+        ab = measure_prefill(M, w, dims, dev, stream, args.seed, chunk=chunk, iters=3)
+        nv = measure_prefill_naive(w, dev, stream, args.seed, chunk)
+        rows.append({"chunk": chunk, "absorbed_us": ab["time_us"], "absorbed_flops": ab["flops"],
+                     "naive": nv})
+        torch.cuda.empty_cache()
+    print(json.dumps({"prefill_forms": rows, "batch": 2, "context": 32768, "heads": w.n_heads}), flush=True)
+
+
 def measure_query_proj(M, w: W.Workload, dims, dev, stream, seed: int, iters: int = 50) -> dict:
     """Average device time of mla_query_proj (its two launches) with a 256 MB
     buffer rewritten between calls, so that the weights come from HBM each time;
@@ -542,6 +633,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-forms", action="store_true",
+                    help="only compare the absorbed and the decompressing prefill forms (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -550,6 +643,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     w = W.WORKLOADS[args.workload]
+    if args.prefill_forms:
+        if rank == 0:
+            prefill_forms(args, w)
+        return
 
     if args.impl == "reference":
         if rank != 0:

@@ -161,6 +161,15 @@ int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
   mla::AbsorbArgs a;
   a.q = q; a.pos = pos; a.w_uk = w_uk; a.q_lat = q_lat; a.n_tokens = n_tokens;
   a.n_heads = dims->n_heads; a.qk_nope = dims->qk_nope; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
+  // each CTA stages one head's W_UK (one CTA per SM fits) and loops over a run of
+  // 16-token blocks: as many CTAs per head as fit in one wave, so that W_UK is
+  // read about once per such CTA instead of once per block
+  int sms = 0;
+  if ((st = device_sms(&sms)) != MLA_OK) return st;
+  const int blocks = (n_tokens + 15) / 16;
+  int per_head = sms / dims->n_heads;
+  if (per_head < 1) per_head = 1;
+  a.blocks_per_cta = (blocks + per_head - 1) / per_head;
   mla::rope_inv_freq(a.inv_freq, dims->d_rope, eff_theta(dims));
   return cuda_status(mla::launch_absorb_q(a, (cudaStream_t)stream));
 }

@@ -158,10 +158,11 @@ __device__ __forceinline__ void absorb_rope_part(const AbsorbArgs& a, int h, int
   }
 }
 
-// q~ = W_UK,h^T q_nope on the tensor cores, one CTA per (head, 16 tokens):
-// D^T [16 tokens x d_c] = Q [16 x qk_nope] . W_UK,h [qk_nope x d_c].  W_UK,h is
-// staged in shared memory (rows padded by 16 bytes) and read as B fragments with
-// ldmatrix.trans; each of the 8 warps owns d_c / 8 output columns.
+// q~ = W_UK,h^T q_nope on the tensor cores, one CTA per (head, run of
+// blocks_per_cta 16-token blocks): per block D^T [16 tokens x d_c] = Q [16 x
+// qk_nope] . W_UK,h [qk_nope x d_c].  W_UK,h is staged in shared memory once
+// (rows padded by 16 bytes) and read as B fragments with ldmatrix.trans; each of
+// the 8 warps owns d_c / 8 output columns.
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -172,7 +173,6 @@ __global__ void __launch_bounds__(kAbsThreads)
 absorb_q_mma_kernel(AbsorbArgs a) {
   extern __shared__ __align__(16) uint16_t wsm[];   // [qk_nope][d_c + 8]
   const int h = blockIdx.x;
-  const int t0 = blockIdx.y * kTokBlk;
   const int dq = a.qk_nope + a.d_rope;
   const int R = a.d_c + a.d_rope;
   const int ws = a.d_c + 8;
@@ -192,8 +192,12 @@ absorb_q_mma_kernel(AbsorbArgs a) {
   // the stream finishes (as in the append kernel above).
   grid_dependency_wait();   // q may be written by the preceding kernel
   allow_dependent_launch();
+  const int nblk = (a.n_tokens + kTokBlk - 1) / kTokBlk;
+  const int blk_end = min(nblk, ((int)blockIdx.y + 1) * a.blocks_per_cta);
+  for (int blk = blockIdx.y * a.blocks_per_cta; blk < blk_end; ++blk) {
+  const int t0 = blk * kTokBlk;
   // A fragments (q_nope of this warp's 16 tokens) for every k step, loaded once
-  // while W_UK,h streams in
+  // per block (the first while W_UK,h streams in)
   const int ta = t0 + g, tb = t0 + g + 8;
   const uint16_t* qa = a.q + ((size_t)ta * a.n_heads + h) * dq;
   const uint16_t* qb = a.q + ((size_t)tb * a.n_heads + h) * dq;
@@ -210,8 +214,10 @@ absorb_q_mma_kernel(AbsorbArgs a) {
     af[k][3] = (kin && vb) ? *reinterpret_cast<const uint32_t*>(qb + ia + 8) : 0u;
   }
   absorb_rope_part(a, h, t0);
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();
+  if (blk == blockIdx.y * a.blocks_per_cta) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+  }
   const int ntiles = a.d_c / 8;
   for (int nt0 = warp * 2; nt0 < ntiles; nt0 += 16) {  // pairs of 8-column tiles
     float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -238,6 +244,7 @@ absorb_q_mma_kernel(AbsorbArgs a) {
       if (vb) *reinterpret_cast<uint32_t*>(a.q_lat + ((size_t)tb * a.n_heads + h) * R + j) = pack_bf16x2(d[n][2], d[n][3]);
     }
   }
+  }   // token blocks
 }
 
 // CUDA-core fallback for shapes whose W_UK,h does not fit in shared memory.
@@ -305,7 +312,9 @@ cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream) {
-  dim3 grid(a.n_heads, (a.n_tokens + kTokBlk - 1) / kTokBlk);
+  const int nblk = (a.n_tokens + kTokBlk - 1) / kTokBlk;
+  const int per = a.blocks_per_cta < 1 ? 1 : a.blocks_per_cta;
+  dim3 grid(a.n_heads, (nblk + per - 1) / per);
   const size_t wsmem = (size_t)a.qk_nope * (a.d_c + 8) * 2;
   cudaLaunchAttribute attr[1] = {pdl_attribute()};
   cudaLaunchConfig_t cfg = {};
@@ -328,6 +337,7 @@ cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(absorb_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
+  cfg.gridDim = dim3(a.n_heads, nblk, 1);   // one 16-token block per CTA
   cfg.dynamicSmemBytes = smem;
   cudaError_t e = cudaLaunchKernelEx(&cfg, absorb_q_kernel, a);
   if (e != cudaSuccess) return e;

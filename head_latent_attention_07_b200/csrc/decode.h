@@ -69,6 +69,7 @@ struct AbsorbArgs {
   const uint16_t* w_uk;       // [H, d_n, d_c]
   uint16_t* q_lat;            // [T, H, d_c + d_r]
   int n_tokens, n_heads, qk_nope, d_c, d_rope;
+  int blocks_per_cta;         // 16-token blocks each CTA of the tensor-core kernel loops over
   double inv_freq[kMaxRopePairs];
 };
 

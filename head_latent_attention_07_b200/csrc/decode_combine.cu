@@ -7,15 +7,15 @@
 //                                                   attending over latents)
 // Work split: one CTA per (head, group of 16 query tokens) over all d_c latent
 // columns.  Its 512 threads merge the partials (32 per token, each owning 16
-// columns; each partial byte is read once, by one CTA), then 16 warps multiply
-// the merged rows by W_UV,h on the tensor cores (mma.sync, fp32 accumulate,
-// o_lat split into two bf16 terms, hi + lo, which keeps about 16 bits of its
-// mantissa): warp w takes out rows [16 (w mod 8), +16) and half of the latent
-// columns, the two halves summed in shared memory.  Independent accumulators
-// (hi and lo terms, even and odd k slices) keep each mma.sync dependence chain
-// 8 deep.  W_UV,h (a chunk of 128 out rows) is staged in shared memory by
-// cp.async before the kernel waits for the split kernel's partials, so after
-// that wait only the merge, the products and the stores remain.
+// columns; each partial byte is read once, by one CTA) and write the merged
+// rows, split into two bf16 terms (hi + lo, which keep about 16 bits of the
+// fp32 mantissa), as the 32 rows of the B operand of one tcgen05 MMA chain:
+// D[128 out rows x 32] = W_UV,h chunk [128 x d_c] . [hi rows; lo rows]^T, fp32
+// in TMEM, d_c / 16 MMAs issued by one thread.  Four warps read D back (one TMEM
+// lane quarter each: 32 out rows) and store hi + lo.  W_UV,h (a chunk of 128 out
+// rows) is staged in shared memory by cp.async, in the 128-byte swizzled
+// K-major layout the MMA reads, before the kernel waits for the split kernel's
+// partials, so after that wait only the merge, the MMAs and the stores remain.
 //
 // Context split (one call per rank over a window of every sequence's pages):
 // with a.out_lat set, the kernel stops after the merge and writes the rank's
@@ -26,18 +26,36 @@
 #include "decode.h"
 #include "mma_frag.cuh"
 #include "plan.cuh"
+#include "sm100.cuh"
 
 namespace mla {
 
 namespace {
 
+using namespace sm100;
+
 constexpr int kThreads = 512;
 constexpr int kTok = 16;       // query tokens per CTA
 constexpr int kCols = 512;     // latent columns per CTA (d_c <= 512)
 constexpr int kVChunk = 128;   // out rows per round (8 row tiles x 16)
-constexpr int kOStride = kCols + 8;    // bf16 row stride of the merged rows (16-byte pad)
-constexpr int kWStride = kCols + 8;    // bf16 row stride of the staged W_UV rows (16-byte pad)
 constexpr int kPieceBatch = 4;         // pieces whose loads are in flight at once
+// MMA operands in shared memory, K-major, 128-byte swizzle: blocks of 64 latent
+// columns, 128 bytes per row, 16-byte chunk c of row r at chunk c ^ (r mod 8)
+constexpr int kKBlocks = kCols / 64;
+constexpr int kWBlock = kVChunk * 128;        // [128 out rows x 64 columns] of W_UV
+constexpr int kOBlock = 2 * kTok * 128;       // [32 rows (hi, lo) x 64 columns] of the merged rows
+constexpr uint32_t kTmemCols = 32;
+
+// One lane of the (converged) warp returns true.
+__device__ __forceinline__ bool elect_lane() {
+  uint32_t is_leader;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(is_leader));
+  return is_leader != 0;
+}
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return uint32_t(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -47,11 +65,14 @@ template <bool RANKS>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_combine_kernel(DecodeArgs a, const __grid_constant__ RankSources src) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  PlanSmem* ps = reinterpret_cast<PlanSmem*>(smem_raw);
-  uint16_t* o_hi = reinterpret_cast<uint16_t*>(smem_raw + ((sizeof(PlanSmem) + 15) & ~size_t(15)));
-  uint16_t* o_lo = o_hi + kTok * kOStride;
-  float* red = reinterpret_cast<float*>(o_lo + kTok * kOStride);       // [kVChunk][kTok] upper-half products
-  uint16_t* wsm = reinterpret_cast<uint16_t*>(red + kVChunk * kTok);  // [kVChunk][kWStride] W_UV rows
+  // swizzled operand blocks first, on a 1024-byte boundary
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t w_s = smem_addr(sm);                      // kKBlocks x kWBlock
+  const uint32_t o_s = w_s + kKBlocks * kWBlock;           // kKBlocks x kOBlock
+  PlanSmem* ps = reinterpret_cast<PlanSmem*>(sm + kKBlocks * (kWBlock + kOBlock));
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(ps) +
+                                                  ((sizeof(PlanSmem) + 15) & ~size_t(15)));
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_bar + 1);
 
   const int h = blockIdx.x;
   const int t0 = blockIdx.y * kTok;
@@ -61,23 +82,33 @@ decode_combine_kernel(DecodeArgs a, const __grid_constant__ RankSources src) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, q = lane & 3;
   const uint16_t* wh = a.w_uv + (size_t)h * a.v_head * a.d_c;
-  // W_UV,h rows [v0, v0 + kVChunk) -> shared memory (zeros outside the matrix)
+  // W_UV,h rows [v0, v0 + kVChunk) -> the swizzled A operand (zeros outside the matrix)
   auto stage_w = [&](int v0) {
     for (int idx = tid; idx < kVChunk * (kCols / 8); idx += kThreads) {
-      const int vl = idx / (kCols / 8), cc = 8 * (idx % (kCols / 8));
-      uint16_t* dst = wsm + vl * kWStride + cc;
+      const int vl = idx / (kCols / 8), cc8 = idx % (kCols / 8), cc = 8 * cc8;
+      const uint32_t dst = w_s + (cc8 >> 3) * kWBlock + swz(vl, cc8 & 7);
       if (v0 + vl < a.v_head && cc < ncol) {
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)),
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
                      "l"(wh + (size_t)(v0 + vl) * a.d_c + cc)
                      : "memory");
       } else {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-
   const bool lat_mode = !RANKS && a.out_lat != nullptr;
+  if (!lat_mode) {   // the latent form stops after the merge: no MMA, no TMEM
+    if (tid == 0) {
+      mbar_init(mma_bar, 1);
+      fence_mbar_init();
+    }
+    if (warp == 0) {
+      tmem_alloc(tmem_holder, kTmemCols);
+      tmem_relinquish();
+    }
+  }
+
   if (RANKS) {
     // the predecessor is the caller's: only the weight rows are read before the
     // wait (the kernel enqueued just before the call must not write W_UV)
@@ -194,88 +225,77 @@ decode_combine_kernel(DecodeArgs a, const __grid_constant__ RankSources src) {
         hi[e] = pack_bf16x2(x0, x1);
         lo[e] = pack_bf16x2(x0 - bf16_lo(hi[e]), x1 - bf16_hi(hi[e]));
       }
-      const int c0 = 256 * half + 8 * gc;
-      *reinterpret_cast<uint4*>(o_hi + j * kOStride + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(o_lo + j * kOStride + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      const int cc8 = 32 * half + gc;                  // 16-byte chunk of the row
+      const uint32_t blk = o_s + (cc8 >> 3) * kOBlock;
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + swz(j, cc8 & 7)), "r"(hi[0]),
+                   "r"(hi[1]), "r"(hi[2]), "r"(hi[3]) : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + swz(kTok + j, cc8 & 7)), "r"(lo[0]),
+                   "r"(lo[1]), "r"(lo[2]), "r"(lo[3]) : "memory");
     }
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
+  fence_proxy_async_smem();   // operands written by this thread -> the tensor core
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
 
-  // 2. per chunk of 128 out rows: warp w multiplies its 16 rows of W_UV by the
-  //    merged rows over latent half w / 8 (32-wide k slices, see mma_frag.cuh);
-  //    the upper half's products go through shared memory to the lower half's
-  //    warp, which adds them and stores out
-  const int rt = warp & 7, kh = warp >> 3;
-  for (int v0 = 0; v0 < a.v_head; v0 += kVChunk) {
+  // 2. per chunk of 128 out rows: one thread issues the MMA chain over the latent
+  //    columns; warps 0-3 read D (lane = out row, columns = hi and lo of each
+  //    token) and store hi + lo
+  const uint32_t idesc = idesc_bf16_f32(128, 2 * kTok, 0, 0);
+  const int ksteps = (ncol + 15) / 16;
+  bool ok = true;
+  for (int v0 = 0, chunk = 0; v0 < a.v_head; v0 += kVChunk, ++chunk) {
     if (v0 > 0) {
-      __syncthreads();   // every warp is done with the previous chunk's W rows and products
       stage_w(v0);
       asm volatile("cp.async.wait_all;" ::: "memory");
+      fence_proxy_async_smem();
+      tc_fence_before();
       __syncthreads();
+      tc_fence_after();
     }
-    float d[2][2][2][4];   // [token tile][hi, lo term][k slice parity][fragment]
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int tm = 0; tm < 2; ++tm)
-#pragma unroll
-        for (int pa = 0; pa < 2; ++pa)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) d[nt][tm][pa][e] = 0.f;
-    const int va = rt * 16 + g, vb = va + 8;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int k0 = 256 * kh + 32 * u;
-      if (k0 >= ncol) break;                    // the same in every lane of the warp
-      const int kk = k0 + 8 * q;
-      const uint4 wa = *reinterpret_cast<const uint4*>(wsm + va * kWStride + kk);
-      const uint4 wb = *reinterpret_cast<const uint4*>(wsm + vb * kWStride + kk);
-      const uint4 h0 = *reinterpret_cast<const uint4*>(o_hi + g * kOStride + kk);
-      const uint4 l0 = *reinterpret_cast<const uint4*>(o_lo + g * kOStride + kk);
-      const uint4 h1 = *reinterpret_cast<const uint4*>(o_hi + (g + 8) * kOStride + kk);
-      const uint4 l1 = *reinterpret_cast<const uint4*>(o_lo + (g + 8) * kOStride + kk);
-      mma_k32(d[0][0][u & 1], wa, wb, h0);
-      mma_k32(d[0][1][u & 1], wa, wb, l0);
-      mma_k32(d[1][0][u & 1], wa, wb, h1);
-      mma_k32(d[1][1][u & 1], wa, wb, l1);
-    }
-    // D fragment: (row g | g+8, token column 2q | 2q+1) of each 8-token tile
-    float dd[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        dd[nt][e] = (d[nt][0][0][e] + d[nt][0][1][e]) + (d[nt][1][0][e] + d[nt][1][1][e]);
-    if (kh == 1) {
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          red[(rt * 16 + g + ((e & 2) ? 8 : 0)) * kTok + nt * 8 + 2 * q + (e & 1)] = dd[nt][e];
-    }
-    __syncthreads();
-    if (kh == 0) {
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int vl = rt * 16 + g + ((e & 2) ? 8 : 0);
-          const int tl = nt * 8 + 2 * q + (e & 1);
-          const int v = v0 + vl, t = t0 + tl;
-          if (v < a.v_head && t < T)
-            a.out[((size_t)t * a.n_heads + h) * a.v_head + v] = f32_to_bf16(dd[nt][e] + red[vl * kTok + tl]);
+    if (warp == 0) {
+      if (elect_lane()) {
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint32_t kb = ks >> 2, k4 = ks & 3;
+          const uint64_t da = smem_desc(w_s + kb * kWBlock + k4 * 32, 16, 1024, kSwizzle128);
+          const uint64_t db = smem_desc(o_s + kb * kOBlock + k4 * 32, 16, 1024, kSwizzle128);
+          mma_bf16(tmem, da, db, idesc, ks > 0 ? 1u : 0u);
         }
+        mma_commit(mma_bar);
+      }
+      __syncwarp();
     }
+    if (warp < 4) {
+      // D complete: a bounded wait (the MMAs of this CTA only)
+      ok = mbar_wait_drain(mma_bar, chunk & 1, 1ll << 31);
+      if (!ok && lane == 0) record_status(a.dev_status, MLA_ERR_TIMEOUT);
+      tc_fence_after();
+      float dv[32];
+      tmem_ld32(tmem + (uint32_t(warp * 32) << 16), dv);
+      tmem_wait_ld();
+      const int v = v0 + warp * 32 + lane;
+      if (ok && v < a.v_head) {
+#pragma unroll
+        for (int tl = 0; tl < kTok; ++tl) {
+          const int t = t0 + tl;
+          if (t < T) a.out[((size_t)t * a.n_heads + h) * a.v_head + v] = f32_to_bf16(dv[tl] + dv[kTok + tl]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();   // D read and the A operand free before the next chunk's MMAs
+    tc_fence_after();
   }
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
 
 size_t decode_combine_smem_bytes(int d_c) {
   (void)d_c;
-  return ((sizeof(PlanSmem) + 15) & ~size_t(15)) + 2ull * kTok * kOStride * 2 + (size_t)kVChunk * kTok * 4 +
-         (size_t)kVChunk * kWStride * 2;
+  return 1024 + (size_t)kKBlocks * (kWBlock + kOBlock) + ((sizeof(PlanSmem) + 15) & ~size_t(15)) + 64;
 }
 
 namespace {
