@@ -2,10 +2,11 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3] [--impl ours|reference]
 
-A step is the whole hot path for one layer: mla_append_latent (this step's
-cache rows), mla_absorb_q and mla_decode_attn (split-KV attention, LSE
-combine, W_UV) over a batch of synthetic sequences whose latent cache is
-resident in HBM.  The default workload is DeepSeek-V3-shaped decode: 16
+A step is the whole hot path for one layer: this step's cache rows and
+absorbed queries (mla_append_absorb: mla_append_latent and mla_absorb_q in one
+launch; the two calls in turn above 16 tokens), then mla_decode_attn (split-KV
+attention, LSE combine, W_UV) over a batch of synthetic sequences whose latent
+cache is resident in HBM.  The default workload is DeepSeek-V3-shaped decode: 16
 sequences, 128 heads, context 32768, 64-token pages, shuffled page table.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
@@ -245,12 +246,23 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
         M.mla_decode_attn(dims, q_lat, pool, page_table, seq_lens_, w_uv, ws, out, lse, dev_status=status,
                           stream=stream)
 
+    # the step's append and absorb (the same tokens and positions) in one call
+    fused = T <= 16 and np.array_equal(x.h_pos, x.pos) and np.array_equal(x.h_seq_idx, x.seq_idx)
+
+    def prologue_(h_, q_, seq_idx_, pos_):
+        if fused:
+            M.mla_append_absorb(dims, h_, w_dkv, seq_idx_, pos_, page_table, pool, q_, w_uk,
+                                q_lat.view(T, w.n_heads, w.row), dev_status=status, stream=stream)
+        else:
+            append_(h_, seq_idx_, pos_)
+            absorb_(q_, pos_)
+
     def step(h_, q_, seq_idx_, pos_, seq_lens_):
-        append_(h_, seq_idx_, pos_)
-        absorb_(q_, pos_)
+        prologue_(h_, q_, seq_idx_, pos_)
         decode_(seq_lens_)
 
-    launches_per_step = 4  # append, absorb, decode split, decode combine
+    # append + absorb (one launch when fused), decode split, decode combine
+    launches_per_step = 3 if fused else 4
 
     def barrier():
         if world > 1:
@@ -295,6 +307,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
     decode_ms = timed(lambda: decode_(seq_lens), n_phase) / n_phase
     append_ms = timed(lambda: append_(h, seq_idx, pos), n_phase) / n_phase
     absorb_ms = timed(lambda: absorb_(q, pos), n_phase) / n_phase
+    prologue_ms = timed(lambda: prologue_(h, q, seq_idx, pos), n_phase) / n_phase
     hot_ms = None
     if flushed:   # the same steps back to back with the cache hot in L2
         flushed = False
@@ -337,9 +350,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
             if i >= 2:
                 stream.wait_event(out_read[i - 2])           # outs[i % 2] has been copied out
             b = dbuf[i % 2]
-            M.mla_append_latent(dims, b["h"], w_dkv, b["seq_idx"], b["pos"], page_table, pool, dev_status=status,
-                                stream=stream)
-            M.mla_absorb_q(dims, b["q"], b["pos"], w_uk, q_lat.view(T, w.n_heads, w.row), stream=stream)
+            prologue_(b["h"], b["q"], b["seq_idx"], b["pos"])
             M.mla_decode_attn(dims, q_lat, pool, page_table, b["seq_lens"], w_uv, ws, outs[i % 2], lse,
                               dev_status=status, stream=stream)
             done[i].record(stream)
@@ -372,9 +383,7 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
             b = dbuf[i % 2]
             for k in host:
                 b[k].copy_(host[k], non_blocking=True)
-            M.mla_append_latent(dims, b["h"], w_dkv, b["seq_idx"], b["pos"], page_table, pool, dev_status=status,
-                                stream=stream)
-            M.mla_absorb_q(dims, b["q"], b["pos"], w_uk, q_lat.view(T, w.n_heads, w.row), stream=stream)
+            prologue_(b["h"], b["q"], b["seq_idx"], b["pos"])
             M.mla_decode_attn(dims, q_lat, pool, page_table, b["seq_lens"], w_uv, ws, outs[i % 2], lse,
                               dev_status=status, stream=stream)
             out_host[i % 2].copy_(outs[i % 2], non_blocking=True)
@@ -392,13 +401,14 @@ def run_ours(args, w: W.Workload, rank: int, world: int, local_rank: int):
                  "query_proj": measure_query_proj(M, w, dims, dev, stream, args.seed + rank),
                  "prefill": measure_prefill(M, w, dims, dev, stream, args.seed + rank)}
     keys = sorted(extra)
-    vals = max_over_ranks([ms_total, e2e_ms, decode_ms, append_ms, absorb_ms, hot_ms or 0.0]
+    vals = max_over_ranks([ms_total, e2e_ms, decode_ms, append_ms, absorb_ms, prologue_ms, hot_ms or 0.0]
                           + [extra[k]["time_us"] for k in keys], dev)
-    ms_total, e2e_ms, decode_ms, append_ms, absorb_ms, hot_ms2 = vals[:6]
-    for k, v in zip(keys, vals[6:]):
+    ms_total, e2e_ms, decode_ms, append_ms, absorb_ms, prologue_ms, hot_ms2 = vals[:7]
+    for k, v in zip(keys, vals[7:]):
         extra[k]["time_us"] = v
     return {"ms_total": ms_total, "e2e_ms": e2e_ms, "decode_ms": decode_ms, "decode_loop_ms": decode_ms * n_phase,
-            "phases_ms": {"append": append_ms, "absorb": absorb_ms, "decode": decode_ms},
+            "phases_ms": {"append": append_ms, "absorb": absorb_ms,
+                          ("append_absorb" if fused else "append_then_absorb"): prologue_ms, "decode": decode_ms},
             "hot_ms": hot_ms2 if hot_ms is not None else None, "clocks": clocks,
             "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "lens": x.lens, **extra}
 

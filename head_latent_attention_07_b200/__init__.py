@@ -12,6 +12,7 @@ importing the binding fails loudly when the shared library has not been built.
     mla.mla_query_proj(dims, h, w_dq, w_uq, c_q, q)          # q-LoRA query path (optional)
     mla.mla_append_latent(dims, h, w_dkv, seq_idx, pos, page_table, pool)
     mla.mla_absorb_q(dims, q, pos, w_uk, q_lat)
+    # or both in one launch: mla.mla_append_absorb(dims, h, w_dkv, seq_idx, pos, page_table, pool, q, w_uk, q_lat)
     mla.mla_decode_attn(dims, q_lat, pool, page_table, seq_lens, w_uv, workspace, out, lse)
     mla.mla_out_proj(dims, out, w_o, y)                       # layer output (optional)
 
@@ -41,6 +42,7 @@ _I = ctypes.c_int32
 SIGNATURES = {
     "mla_append_latent": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _P, _P]),
     "mla_absorb_q": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _P]),
+    "mla_append_absorb": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _I, _P, _P]),
     "mla_decode_workspace_bytes": (ctypes.c_size_t, [_P, _I, _I]),
     "mla_decode_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, ctypes.c_size_t,
                                        _P, _P, _P, _P]),
@@ -186,6 +188,32 @@ def mla_absorb_q(dims: MlaDims, q, pos, w_uk, q_lat, stream=None) -> None:
         ctypes.byref(dims), _ptr(q, torch.bfloat16, "q"), _ptr(pos, torch.int32, "pos"),
         _ptr(w_uk, torch.bfloat16, "w_uk"), _ptr(q_lat, torch.bfloat16, "q_lat"), T, _stream(stream))
     _check(st, "mla_absorb_q")
+
+
+def mla_append_absorb(dims: MlaDims, h, w_dkv, seq_idx, pos, page_table, pool, q, w_uk, q_lat,
+                      dev_status=None, stream=None) -> None:
+    """mla_append_latent and mla_absorb_q of one decode step (the same tokens and
+    positions) in one call."""
+    torch = _torch()
+    T = h.shape[0]
+    B, max_pages = page_table.shape
+    num_pages = pool.shape[0]
+    _shape(h, (T, dims.d_model), "h")
+    _shape(w_dkv, (dims.row, dims.d_model), "w_dkv")
+    _shape(seq_idx, (T,), "seq_idx")
+    _shape(pos, (T,), "pos")
+    _shape(pool, (num_pages, dims.page_size, dims.row), "pool")
+    _shape(q, (T, dims.n_heads, dims.qk_nope + dims.d_rope), "q")
+    _shape(w_uk, (dims.n_heads, dims.qk_nope, dims.d_c), "w_uk")
+    _shape(q_lat, (T, dims.n_heads, dims.row), "q_lat")
+    st = load_library().mla_append_absorb(
+        ctypes.byref(dims), _ptr(h, torch.bfloat16, "h"), _ptr(w_dkv, torch.bfloat16, "w_dkv"),
+        _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(pos, torch.int32, "pos"),
+        _ptr(page_table, torch.int32, "page_table"), B, max_pages,
+        _ptr(pool, torch.bfloat16, "pool"), num_pages, _ptr(q, torch.bfloat16, "q"),
+        _ptr(w_uk, torch.bfloat16, "w_uk"), _ptr(q_lat, torch.bfloat16, "q_lat"), T,
+        _ptr(dev_status, torch.int32, "dev_status"), _stream(stream))
+    _check(st, "mla_append_absorb")
 
 
 def mla_decode_workspace_bytes(dims: MlaDims, batch: int, nq: int) -> int:

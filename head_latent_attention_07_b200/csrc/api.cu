@@ -126,12 +126,12 @@ namespace mla {
 int record_cuda_error(cudaError_t e) { return cuda_status(e); }
 }  // namespace mla
 
-extern "C" {
+namespace {
 
-int mla_append_latent(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv,
-                      const int32_t* seq_idx, const int32_t* pos, const int32_t* page_table,
-                      int32_t batch, int32_t max_pages, mla_bf16* pool, int32_t num_pages,
-                      int32_t n_tokens, int32_t* dev_status, void* stream) {
+// Checks and fills the arguments of mla_append_latent (also for mla_append_absorb).
+int append_args(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv, const int32_t* seq_idx,
+                const int32_t* pos, const int32_t* page_table, int32_t batch, int32_t max_pages, mla_bf16* pool,
+                int32_t num_pages, int32_t n_tokens, int32_t* dev_status, mla::AppendArgs* a) {
   int st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (n_tokens < 0 || batch < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
@@ -141,26 +141,25 @@ int mla_append_latent(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w
       !aligned16(page_table) || !aligned16(pool) || (dev_status && !aligned16(dev_status)))
     return MLA_ERR_MISALIGNED;
   if ((int64_t)max_pages * dims->page_size > INT32_MAX) return MLA_ERR_UNSUPPORTED;
-  mla::AppendArgs a;
-  a.h = h; a.w_dkv = w_dkv; a.seq_idx = seq_idx; a.pos = pos; a.page_table = page_table;
-  a.pool = pool; a.dev_status = dev_status; a.n_tokens = n_tokens; a.d_model = dims->d_model;
-  a.d_c = dims->d_c; a.d_rope = dims->d_rope; a.page_size = dims->page_size; a.batch = batch;
-  a.max_pages = max_pages; a.num_pages = num_pages;
-  mla::rope_inv_freq(a.inv_freq, dims->d_rope, eff_theta(dims));
-  return cuda_status(mla::launch_append_latent(a, (cudaStream_t)stream));
+  a->h = h; a->w_dkv = w_dkv; a->seq_idx = seq_idx; a->pos = pos; a->page_table = page_table;
+  a->pool = pool; a->dev_status = dev_status; a->n_tokens = n_tokens; a->d_model = dims->d_model;
+  a->d_c = dims->d_c; a->d_rope = dims->d_rope; a->page_size = dims->page_size; a->batch = batch;
+  a->max_pages = max_pages; a->num_pages = num_pages;
+  mla::rope_inv_freq(a->inv_freq, dims->d_rope, eff_theta(dims));
+  return MLA_OK;
 }
 
-int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
-                 const mla_bf16* w_uk, mla_bf16* q_lat, int32_t n_tokens, void* stream) {
+// Checks and fills the arguments of mla_absorb_q (also for mla_append_absorb).
+int absorb_args(const mla_dims* dims, const mla_bf16* q, const int32_t* pos, const mla_bf16* w_uk,
+                mla_bf16* q_lat, int32_t n_tokens, mla::AbsorbArgs* a) {
   int st = check_dims(dims);
   if (st != MLA_OK) return st;
   if (n_tokens < 0) return MLA_ERR_INVALID_ARG;
   if (n_tokens == 0) return MLA_OK;
   if (!q || !pos || !w_uk || !q_lat) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(pos) || !aligned16(w_uk) || !aligned16(q_lat)) return MLA_ERR_MISALIGNED;
-  mla::AbsorbArgs a;
-  a.q = q; a.pos = pos; a.w_uk = w_uk; a.q_lat = q_lat; a.n_tokens = n_tokens;
-  a.n_heads = dims->n_heads; a.qk_nope = dims->qk_nope; a.d_c = dims->d_c; a.d_rope = dims->d_rope;
+  a->q = q; a->pos = pos; a->w_uk = w_uk; a->q_lat = q_lat; a->n_tokens = n_tokens;
+  a->n_heads = dims->n_heads; a->qk_nope = dims->qk_nope; a->d_c = dims->d_c; a->d_rope = dims->d_rope;
   // each CTA stages one head's W_UK (one CTA per SM fits) and loops over a run of
   // 16-token blocks: as many CTAs per head as fit in one wave, so that W_UK is
   // read about once per such CTA instead of once per block
@@ -169,9 +168,46 @@ int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
   const int blocks = (n_tokens + 15) / 16;
   int per_head = sms / dims->n_heads;
   if (per_head < 1) per_head = 1;
-  a.blocks_per_cta = (blocks + per_head - 1) / per_head;
-  mla::rope_inv_freq(a.inv_freq, dims->d_rope, eff_theta(dims));
+  a->blocks_per_cta = (blocks + per_head - 1) / per_head;
+  mla::rope_inv_freq(a->inv_freq, dims->d_rope, eff_theta(dims));
+  return MLA_OK;
+}
+
+}  // namespace
+
+
+extern "C" {
+
+int mla_append_latent(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv,
+                      const int32_t* seq_idx, const int32_t* pos, const int32_t* page_table,
+                      int32_t batch, int32_t max_pages, mla_bf16* pool, int32_t num_pages,
+                      int32_t n_tokens, int32_t* dev_status, void* stream) {
+  mla::AppendArgs a;
+  const int st = append_args(dims, h, w_dkv, seq_idx, pos, page_table, batch, max_pages, pool, num_pages, n_tokens,
+                             dev_status, &a);
+  if (st != MLA_OK || n_tokens == 0) return st;
+  return cuda_status(mla::launch_append_latent(a, (cudaStream_t)stream));
+}
+
+int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
+                 const mla_bf16* w_uk, mla_bf16* q_lat, int32_t n_tokens, void* stream) {
+  mla::AbsorbArgs a;
+  const int st = absorb_args(dims, q, pos, w_uk, q_lat, n_tokens, &a);
+  if (st != MLA_OK || n_tokens == 0) return st;
   return cuda_status(mla::launch_absorb_q(a, (cudaStream_t)stream));
+}
+
+int mla_append_absorb(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv, const int32_t* seq_idx,
+                      const int32_t* pos, const int32_t* page_table, int32_t batch, int32_t max_pages,
+                      mla_bf16* pool, int32_t num_pages, const mla_bf16* q, const mla_bf16* w_uk,
+                      mla_bf16* q_lat, int32_t n_tokens, int32_t* dev_status, void* stream) {
+  mla::AppendArgs ap;
+  mla::AbsorbArgs ab;
+  int st = append_args(dims, h, w_dkv, seq_idx, pos, page_table, batch, max_pages, pool, num_pages, n_tokens,
+                       dev_status, &ap);
+  if (st != MLA_OK) return st;
+  if ((st = absorb_args(dims, q, pos, w_uk, q_lat, n_tokens, &ab)) != MLA_OK || n_tokens == 0) return st;
+  return cuda_status(mla::launch_append_absorb(ap, ab, (cudaStream_t)stream));
 }
 
 size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t nq) {

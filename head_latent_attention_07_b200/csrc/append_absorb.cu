@@ -140,12 +140,12 @@ append_latent_kernel(AppendArgs a) {
 constexpr int kAbsThreads = 256;
 constexpr int kAbsMaxKSteps = 12;   // tensor-core path: qk_nope <= 192
 
-// RoPE(q_rope, pos) of one head for up to kTokBlk tokens.
-__device__ __forceinline__ void absorb_rope_part(const AbsorbArgs& a, int h, int t0) {
+// RoPE(q_rope, pos) of one head for up to kTokBlk tokens, by threads tid of nthreads.
+__device__ __forceinline__ void absorb_rope_part(const AbsorbArgs& a, int h, int t0, int tid, int nthreads) {
   const int dq = a.qk_nope + a.d_rope;
   const int R = a.d_c + a.d_rope;
   const int npair = a.d_rope / 2;
-  for (int idx = threadIdx.x; idx < kTokBlk * npair; idx += blockDim.x) {
+  for (int idx = tid; idx < kTokBlk * npair; idx += nthreads) {
     const int k = idx / npair, i = idx % npair;
     const int t = t0 + k;
     if (t >= a.n_tokens) continue;
@@ -213,7 +213,7 @@ absorb_q_mma_kernel(AbsorbArgs a) {
     af[k][2] = (kin && va) ? *reinterpret_cast<const uint32_t*>(qa + ia + 8) : 0u;
     af[k][3] = (kin && vb) ? *reinterpret_cast<const uint32_t*>(qb + ia + 8) : 0u;
   }
-  absorb_rope_part(a, h, t0);
+  absorb_rope_part(a, h, t0, threadIdx.x, blockDim.x);
   if (blk == blockIdx.y * a.blocks_per_cta) {
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
@@ -287,7 +287,172 @@ absorb_q_kernel(AbsorbArgs a) {
             pack_bf16x2(acc0[k], acc1[k]);
     }
   }
-  absorb_rope_part(a, h, t0);
+  absorb_rope_part(a, h, t0, threadIdx.x, blockDim.x);
+}
+
+// ------------------------------------------------------------------ append + absorb in one launch
+// A decode step's two prologue calls on the same <= 16 tokens are independent:
+// one launch runs both, so that neither waits for the other.  CTA i < H absorbs
+// head i's queries with warps 0-7 (as absorb_q_mma_kernel, one 16-token block);
+// every CTA also computes with warps 8-15 up to kFusedMaxRows rows of [c || k^]
+// (whole RoPE pairs: the R / 2 pairs are dealt evenly to the CTAs) for all the
+// tokens: 32-wide slices of d_model dealt to the warps (rows g < 8 of the
+// mma.sync tile), the warps' tiles summed in shared memory, then RoPE and the
+// store as in append_latent_kernel.  Weights (W_UK,h and the rows of w_dkv) are
+// read before the dependency wait.
+constexpr int kFusedThreads = 512;
+constexpr int kFusedMaxRows = 8;
+
+__device__ __forceinline__ void role_sync(int id) {
+  asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");   // the 8 warps of one role
+}
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+append_absorb_kernel(AppendArgs ap, AbsorbArgs ab, int npairs) {
+  extern __shared__ __align__(16) uint16_t wsm[];          // absorb: [qk_nope][d_c + 8]
+  __shared__ float part[8][kFusedMaxRows][17];             // append: per warp [row][token]
+  __shared__ float vals[kFusedMaxRows][17];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q4 = lane & 3;
+  const int h = blockIdx.x;
+  const bool absorb_cta = h < ab.n_heads;
+  const int R = ap.d_c + ap.d_rope;
+  const int D = ap.d_model;
+  const int T = ap.n_tokens;
+  const int nslices = (D + 31) / 32;
+  const int p0 = (int)(((long long)npairs * blockIdx.x) / gridDim.x);
+  const int p1 = (int)(((long long)npairs * (blockIdx.x + 1)) / gridDim.x);
+  const int r0 = 2 * p0, nrows = 2 * (p1 - p0);          // <= kFusedMaxRows
+  const int ws = ab.d_c + 8;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+
+  // ---- before the dependency wait: weights only
+  if (warp < 8 && absorb_cta) {
+    const uint16_t* wh = ab.w_uk + (size_t)h * ab.qk_nope * ab.d_c;
+    const int cpr = ab.d_c / 8;
+    for (int idx = threadIdx.x; idx < ab.qk_nope * cpr; idx += 256) {
+      const int i = idx / cpr, cch = idx % cpr;
+      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(wsm + i * ws + cch * 8));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(wh + (size_t)i * ab.d_c + cch * 8)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  const int aw = warp - 8;                                   // append warp 0..7
+  uint4 ra[4];
+  auto load_w = [&](int base) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sl = base + 8 * u;
+      const int kk = 32 * sl + 8 * q4;
+      ra[u] = (sl < nslices && kk < D && g < nrows) ? ldg_stream(ap.w_dkv + (size_t)(r0 + g) * D + kk) : z;
+    }
+  };
+  if (warp >= 8) load_w(aw);
+  grid_dependency_wait();   // h, q, the page table and the pool may be written by the preceding kernel
+  allow_dependent_launch();
+
+  if (warp >= 8) {
+    // ---- append: rows [r0, r0 + nrows) for all T tokens
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int base = aw; base < nslices; base += 32) {
+      uint4 ha[4], hb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int sl = base + 8 * u;
+        const int kk = 32 * sl + 8 * q4;
+        const bool kin = sl < nslices && kk < D;
+        ha[u] = (kin && g < T) ? *reinterpret_cast<const uint4*>(ap.h + (size_t)g * D + kk) : z;
+        hb[u] = (kin && g + 8 < T) ? *reinterpret_cast<const uint4*>(ap.h + (size_t)(g + 8) * D + kk) : z;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        mma_k32(d0, ra[u], z, ha[u]);
+        mma_k32(d1, ra[u], z, hb[u]);
+      }
+      if (base + 32 < nslices) load_w(base + 32);
+    }
+    // fragment: row g, tokens 2 q4 + {0, 1} of each 8-token tile (rows g + 8 are empty)
+    part[aw][g][2 * q4] = d0[0];
+    part[aw][g][2 * q4 + 1] = d0[1];
+    part[aw][g][8 + 2 * q4] = d1[0];
+    part[aw][g][8 + 2 * q4 + 1] = d1[1];
+    role_sync(1);
+    const int at = threadIdx.x - 256;
+    const int rr = at >> 4, j = at & 15;                    // 8 rows x 16 tokens over the first 128 threads
+    if (at < kFusedMaxRows * 16) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) v += part[w][rr][j];
+      vals[rr][j] = v;
+    }
+    role_sync(1);
+    if (at < kFusedMaxRows * 16 && rr < nrows && j < T) {
+      const int row = r0 + rr, t = j;
+      const int seq = ap.seq_idx[t], p = ap.pos[t];
+      bool ok = seq >= 0 && seq < ap.batch && p >= 0 && p < ap.max_pages * ap.page_size;
+      const int page = ok ? ap.page_table[(size_t)seq * ap.max_pages + p / ap.page_size] : -1;
+      ok = ok && page >= 0 && page < ap.num_pages;
+      if (!ok) {
+        record_status(ap.dev_status, MLA_ERR_RANGE);
+      } else {
+        float val = vals[rr][j];
+        if (row >= ap.d_c) {
+          const int qch = row - ap.d_c;                    // channel within the RoPE key
+          float c, sn;
+          rope_cos_sin(p, ap.inv_freq[qch >> 1], &c, &sn);
+          const float x0 = vals[rr & ~1][j], x1 = vals[rr | 1][j];
+          val = (qch & 1) ? x0 * sn + x1 * c : x0 * c - x1 * sn;
+        }
+        ap.pool[((size_t)page * ap.page_size + p % ap.page_size) * R + row] = f32_to_bf16(val);
+      }
+    }
+  } else if (absorb_cta) {
+    // ---- absorb: head h, tokens [0, T)
+    const int dq = ab.qk_nope + ab.d_rope;
+    const uint16_t* qa = ab.q + ((size_t)g * ab.n_heads + h) * dq;
+    const uint16_t* qb = ab.q + ((size_t)(g + 8) * ab.n_heads + h) * dq;
+    const bool va = g < ab.n_tokens, vb = g + 8 < ab.n_tokens;
+    const int nks = ab.qk_nope / 16;
+    uint32_t af[kAbsMaxKSteps][4];
+#pragma unroll
+    for (int k = 0; k < kAbsMaxKSteps; ++k) {
+      const int ia = 16 * k + 2 * q4;
+      const bool kin = k < nks;
+      af[k][0] = (kin && va) ? *reinterpret_cast<const uint32_t*>(qa + ia) : 0u;
+      af[k][1] = (kin && vb) ? *reinterpret_cast<const uint32_t*>(qb + ia) : 0u;
+      af[k][2] = (kin && va) ? *reinterpret_cast<const uint32_t*>(qa + ia + 8) : 0u;
+      af[k][3] = (kin && vb) ? *reinterpret_cast<const uint32_t*>(qb + ia + 8) : 0u;
+    }
+    absorb_rope_part(ab, h, 0, threadIdx.x, 256);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    role_sync(2);
+    const int Rq = ab.d_c + ab.d_rope;
+    const int ntiles = ab.d_c / 8;
+    for (int nt0 = warp * 2; nt0 < ntiles; nt0 += 16) {      // pairs of 8-column tiles
+      float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const int j0 = nt0 * 8;
+#pragma unroll
+      for (int k = 0; k < kAbsMaxKSteps; ++k) {
+        if (k >= nks) break;
+        const int i0 = 16 * k;
+        const int tile = lane >> 3, rr = lane & 7;
+        const int wi = i0 + rr + ((tile & 1) ? 8 : 0);
+        const int wj = j0 + ((tile & 2) ? 8 : 0);
+        uint32_t b[4];
+        ldsm_x4_trans(static_cast<uint32_t>(__cvta_generic_to_shared(wsm + wi * ws + wj)), b);
+        mma_16816(d[0], af[k][0], af[k][1], af[k][2], af[k][3], b[0], b[1]);
+        if (nt0 + 1 < ntiles) mma_16816(d[1], af[k][0], af[k][1], af[k][2], af[k][3], b[2], b[3]);
+      }
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const int j = j0 + 8 * n + 2 * q4;
+        if (nt0 + n >= ntiles) continue;
+        if (va) *reinterpret_cast<uint32_t*>(ab.q_lat + ((size_t)g * ab.n_heads + h) * Rq + j) = pack_bf16x2(d[n][0], d[n][1]);
+        if (vb) *reinterpret_cast<uint32_t*>(ab.q_lat + ((size_t)(g + 8) * ab.n_heads + h) * Rq + j) = pack_bf16x2(d[n][2], d[n][3]);
+      }
+    }
+  }
 }
 
 }  // namespace
@@ -340,6 +505,38 @@ cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream) {
   cfg.gridDim = dim3(a.n_heads, nblk, 1);   // one 16-token block per CTA
   cfg.dynamicSmemBytes = smem;
   cudaError_t e = cudaLaunchKernelEx(&cfg, absorb_q_kernel, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+bool append_absorb_fusable(const AppendArgs& ap, const AbsorbArgs& ab) {
+  const size_t wsmem = (size_t)ab.qk_nope * (ab.d_c + 8) * 2;
+  return ap.n_tokens <= kTokBlk && ab.n_tokens == ap.n_tokens && ab.qk_nope % 16 == 0 &&
+         ab.qk_nope <= 16 * kAbsMaxKSteps && ab.d_c % 8 == 0 && wsmem <= 180 * 1024 &&
+         (ap.d_c + ap.d_rope) % 2 == 0;
+}
+
+cudaError_t launch_append_absorb(const AppendArgs& ap, const AbsorbArgs& ab, cudaStream_t stream) {
+  if (!append_absorb_fusable(ap, ab)) {
+    cudaError_t e = launch_append_latent(ap, stream);
+    if (e != cudaSuccess) return e;
+    return launch_absorb_q(ab, stream);
+  }
+  const int npairs = (ap.d_c + ap.d_rope) / 2;
+  const int need = (npairs + kFusedMaxRows / 2 - 1) / (kFusedMaxRows / 2);   // CTAs with <= 8 rows each
+  const int ctas = ab.n_heads > need ? ab.n_heads : need;
+  const size_t wsmem = (size_t)ab.qk_nope * (ab.d_c + 8) * 2;
+  cudaError_t e = cudaFuncSetAttribute(append_absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas, 1, 1);
+  cfg.blockDim = dim3(kFusedThreads, 1, 1);
+  cfg.dynamicSmemBytes = wsmem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, append_absorb_kernel, ap, ab, npairs);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -116,6 +116,9 @@ int record_cuda_error(cudaError_t e);
 
 cudaError_t launch_append_latent(const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
+// Both of the above in one launch when the token count allows (<= 16 tokens),
+// else the two launches in turn.
+cudaError_t launch_append_absorb(const AppendArgs& ap, const AbsorbArgs& ab, cudaStream_t stream);
 int linear_ksplit(int N, int K, int sms);
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t stream);
 

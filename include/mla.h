@@ -144,6 +144,25 @@ int mla_absorb_q(const mla_dims* dims, const mla_bf16* q, const int32_t* pos,
                  const mla_bf16* w_uk, mla_bf16* q_lat, int32_t n_tokens, void* stream);
 
 /*
+ * mla_append_absorb - mla_append_latent and mla_absorb_q of one decode step in
+ * one call: the step's n_tokens tokens are appended (h, w_dkv, seq_idx, pos,
+ * page_table, pool as in mla_append_latent) and their queries absorbed (q, w_uk,
+ * q_lat as in mla_absorb_q, with the same pos: a decode token's query sits at
+ * the cache index of the row it appends).  The two computations are
+ * independent ([songhuiming] "Step-by-step for t100": the new latent is
+ * appended and the query absorbed before attending); with n_tokens <= 16 they
+ * run in one kernel launch, so neither waits for the other, else as the two
+ * calls in turn.  Results equal those of the two calls up to the order of the
+ * fp32 sums of the append (q_lat bit for bit).  Arguments, errors and the
+ * device status word as in the two calls; n_tokens == 0 is a no-op.
+ */
+int mla_append_absorb(const mla_dims* dims, const mla_bf16* h, const mla_bf16* w_dkv,
+                      const int32_t* seq_idx, const int32_t* pos, const int32_t* page_table,
+                      int32_t batch, int32_t max_pages, mla_bf16* pool, int32_t num_pages,
+                      const mla_bf16* q, const mla_bf16* w_uk, mla_bf16* q_lat, int32_t n_tokens,
+                      int32_t* dev_status, void* stream);
+
+/*
  * mla_decode_workspace_bytes - device workspace mla_decode_attn needs for
  * `batch` sequences with `nq` query tokens each, on the current device.
  * Returns 0 for invalid arguments.
