@@ -99,6 +99,7 @@ struct PairParams {
 
 struct Bars {
   uint64_t kfull[2];    // CTA 0: both CTAs' pages of a step landed in the step buffer (2 arrivals + bytes)
+  uint64_t buf_lo[2];   // both: the step's value MMAs are done with blocks 0-3 of its buffer
   uint64_t buf_free[2]; // both: the step's value MMAs are done with its buffer
   uint64_t vland[2];    // local: per-thread peer-half copies of a partial step have landed (32 arrivals)
   uint64_t vfull[2];    // CTA 0: both CTAs' step buffers hold the value operand (2 arrivals)
@@ -234,6 +235,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->kfull[s], 2);
+      mbar_init(&bar->buf_lo[s], 1);
       mbar_init(&bar->buf_free[s], 1);
       mbar_init(&bar->vland[s], 32);
       mbar_init(&bar->vfull[s], 2);
@@ -296,15 +298,23 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         }
       }
       const int u = t & 1;
-      // the value MMAs of step t - 2 must be done with this buffer
-      if (t >= 2 && !wwait(&bar->buf_free[u], ((t >> 1) - 1) & 1)) break;
+      // the value MMAs of step t - 2 must be done with this buffer: blocks 0-3
+      // (latent columns [0,256)) are free once the first half of them is done, so
+      // their loads start before the second half completes
+      int y = 0;
       if (lane == 0) {
         const int id = (int)c < st.np ? page_id(a, st.b, st.pg0 + (int)c, status) : -1;
-        const int y = id >= 0 ? id * 64 : oob_row;
-        unsigned char* dst = buf_s + u * kBufBytes;
-        mbar_arrive_expect_tx_cluster(kfull0 + 8 * u, kBufBytes);
-        for (int blk = 0; blk < 9; ++blk) tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+        y = id >= 0 ? id * 64 : oob_row;
       }
+      unsigned char* dst = buf_s + u * kBufBytes;
+      if (t >= 2 && !wwait(&bar->buf_lo[u], ((t >> 1) - 1) & 1)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx_cluster(kfull0 + 8 * u, kBufBytes);
+        for (int blk = 0; blk < 4; ++blk) tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+      }
+      if (t >= 2 && !wwait(&bar->buf_free[u], ((t >> 1) - 1) & 1)) break;
+      if (lane == 0)
+        for (int blk = 4; blk < 9; ++blk) tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
       ++t;
     }
   } else if (warp == 2) {
@@ -467,6 +477,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 const uint64_t db = smem_desc(bu + (4 * j + 2 * pg) * kBlockBytes + ks * 2048, kBlockBytes, 1024,
                                               kSwizzle128);
                 mma_bf16_pair(tmem + kTmemO + 128 * j, da, db, id_v, (st.first && pg == 0 && ks == 0) ? 0u : 1u);
+                if (j == 0 && pg == 1 && ks == 3) mma_commit_pair(&bar->buf_lo[t & 1]);
               }
           mma_commit_pair(&bar->p_empty[t & 1]);
           mma_commit_pair(&bar->buf_free[t & 1]);
