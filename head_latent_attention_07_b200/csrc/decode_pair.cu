@@ -310,11 +310,17 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
       if (t >= 2 && !wwait(&bar->buf_lo[u], ((t >> 1) - 1) & 1)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx_cluster(kfull0 + 8 * u, kBufBytes);
-        for (int blk = 0; blk < 4; ++blk) tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+        for (int k = 0; k < 5; ++k) {             // blocks 0, 1, 4, 5, 8
+          const int blk = k == 4 ? 8 : (k & 1) + 4 * (k >> 1);
+          tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+        }
       }
       if (t >= 2 && !wwait(&bar->buf_free[u], ((t >> 1) - 1) & 1)) break;
       if (lane == 0)
-        for (int blk = 4; blk < 9; ++blk) tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+        for (int k = 0; k < 4; ++k) {             // blocks 2, 3, 6, 7
+          const int blk = 2 + (k & 1) + 4 * (k >> 1);
+          tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+        }
       ++t;
     }
   } else if (warp == 2) {
@@ -465,9 +471,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         tc_fence_after();
         if (elect_one()) {
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
+          for (int pg = 0; pg < 2; ++pg)
 #pragma unroll
-            for (int pg = 0; pg < 2; ++pg)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks) {      // 16 keys of page pg per MMA
                 // P of page 0 sits in the step buffer's rope block, free once the
@@ -477,7 +483,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                 const uint64_t db = smem_desc(bu + (4 * j + 2 * pg) * kBlockBytes + ks * 2048, kBlockBytes, 1024,
                                               kSwizzle128);
                 mma_bf16_pair(tmem + kTmemO + 128 * j, da, db, id_v, (st.first && pg == 0 && ks == 0) ? 0u : 1u);
-                if (j == 0 && pg == 1 && ks == 3) mma_commit_pair(&bar->buf_lo[t & 1]);
+                // page 0's value blocks (0, 1, 4, 5) and its P (block 8) are done
+                if (pg == 0 && j == 1 && ks == 3) mma_commit_pair(&bar->buf_lo[t & 1]);
               }
           mma_commit_pair(&bar->p_empty[t & 1]);
           mma_commit_pair(&bar->buf_free[t & 1]);
