@@ -29,7 +29,9 @@
 //           page's columns [256j + 128c, +128), read from L2 by TMA (the peer just
 //           loaded that page); where a page is partial, per-thread copies fill slots
 //           past the sequence's end with zeros instead.  So each CTA reads 72 KB per
-//           step from HBM and 32 KB from L2.
+//           step from HBM and 32 KB from L2.  The value MMAs run page by page; once
+//           page 0's are done, the blocks they read (0, 1, 4, 5 and 8) are reloaded
+//           for the step two ahead, the other four when page 1's are done.
 //
 // TMEM (512 columns, same map in both CTAs; a pair tile with M = 128 folds each
 // CTA's 64 rows into the 128 lanes: lanes [0,64) hold the first N/2 columns, lanes
@@ -99,7 +101,7 @@ struct PairParams {
 
 struct Bars {
   uint64_t kfull[2];    // CTA 0: both CTAs' pages of a step landed in the step buffer (2 arrivals + bytes)
-  uint64_t buf_lo[2];   // both: the step's value MMAs are done with blocks 0-3 of its buffer
+  uint64_t buf_lo[2];   // both: the step's value MMAs of page 0 are done (blocks 0, 1, 4, 5, 8 of its buffer)
   uint64_t buf_free[2]; // both: the step's value MMAs are done with its buffer
   uint64_t vland[2];    // local: per-thread peer-half copies of a partial step have landed (32 arrivals)
   uint64_t vfull[2];    // CTA 0: both CTAs' step buffers hold the value operand (2 arrivals)
@@ -298,9 +300,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         }
       }
       const int u = t & 1;
-      // the value MMAs of step t - 2 must be done with this buffer: blocks 0-3
-      // (latent columns [0,256)) are free once the first half of them is done, so
-      // their loads start before the second half completes
+      // the value MMAs of step t - 2 must be done with this buffer: the blocks
+      // they read for page 0 (0, 1, 4, 5 and block 8, page 0's P) are free once
+      // those MMAs are done, so their loads start before the page-1 MMAs complete
       int y = 0;
       if (lane == 0) {
         const int id = (int)c < st.np ? page_id(a, st.b, st.pg0 + (int)c, status) : -1;
