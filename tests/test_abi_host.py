@@ -94,6 +94,26 @@ def test_append_argument_checks(lib):
     assert call(T=0, h=None) == M.MLA_OK
 
 
+def test_append_absorb_argument_checks(lib):
+    # the checks of both calls it stands for, before any launch
+    d = v3_dims()
+    call = lambda dims=d, **kw: lib.mla_append_absorb(
+        ctypes.byref(dims) if dims is not None else None, kw.get("h", FAKE), FAKE, FAKE, kw.get("pos", FAKE),
+        FAKE, kw.get("B", 2), 4, kw.get("pool", FAKE), 8, kw.get("q", FAKE), FAKE, kw.get("q_lat", FAKE),
+        kw.get("T", 2), kw.get("st", None), None)
+    assert call(dims=None) == M.MLA_ERR_INVALID_ARG
+    assert call(dims=v3_dims(d_rope=0)) == M.MLA_ERR_UNSUPPORTED
+    assert call(h=None) == M.MLA_ERR_INVALID_ARG
+    assert call(q=None) == M.MLA_ERR_INVALID_ARG
+    assert call(q_lat=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(pool=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(pos=FAKE_MIS) == M.MLA_ERR_MISALIGNED
+    assert call(st=FAKE + 4) == M.MLA_ERR_MISALIGNED
+    assert call(B=0) == M.MLA_ERR_INVALID_ARG
+    assert call(T=-1) == M.MLA_ERR_INVALID_ARG
+    assert call(T=0, h=None, q=None) == M.MLA_OK                      # empty: no-op
+
+
 def test_decode_argument_checks(lib):
     d = v3_dims()
     def call(**kw):
