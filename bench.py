@@ -32,7 +32,9 @@ the step's output) and the q-LoRA query path c_Q = W_DQ h, q = W_UQ c_Q
 (mla_query_proj, q_lora_rank 1536), each timed alone after the step (neither is
 part of the step); W_O (235 MB at the V3 shape) is larger than L2, W_DQ + W_UQ
 (97.5 MB) are not, so an L2-sized buffer is rewritten before each timed call of
-the query path.  next_rows.prefill: mla_decode_attn on a chunk of 128 new tokens
+the query path (query_proj.layers_back_to_back: the same calls back to back, each
+with another layer's copy of the weights, the copies together over twice the
+L2).  next_rows.prefill: mla_decode_attn on a chunk of 128 new tokens
 per sequence (2 sequences of 32768, V3 heads), compute-bound, against the bf16
 tensor peak.
 
@@ -536,7 +538,10 @@ def prefill_forms(args, w: W.Workload) -> None:
 def measure_query_proj(M, w: W.Workload, dims, dev, stream, seed: int, iters: int = 50) -> dict:
     """Average device time of mla_query_proj (its two launches) with a 256 MB
     buffer rewritten between calls, so that the weights come from HBM each time;
-    each call is bracketed by its own CUDA events on the launching stream."""
+    each call is bracketed by its own CUDA events on the launching stream.  Also
+    the average over back-to-back calls that take, in turn, the weights of as many
+    layers (copies) as exceed twice the L2: the weights again come from HBM, and
+    each call overlaps its neighbours as a model's layers would."""
     import torch
     r = W.Q_LORA_RANK
     x = W.make_query_proj_inputs(w, seed, w.tokens, r)
@@ -558,7 +563,24 @@ def measure_query_proj(M, w: W.Workload, dims, dev, stream, seed: int, iters: in
     torch.cuda.synchronize(dev)
     us = float(np.mean([a.elapsed_time(b) for a, b in times])) * 1000.0
     nbytes = (w_dq.numel() + w_uq.numel() + h.numel() + 2 * c_q.numel() + q.numel()) * 2
+    # as a model's layers run it: back-to-back calls, each with another layer's
+    # weights (copies whose total exceeds twice the L2), no flush in between
+    layers = max(2, -(-2 * L2_BYTES // ((w_dq.numel() + w_uq.numel()) * 2)) + 1)
+    mats = [(w_dq, w_uq)] + [(w_dq.clone(), w_uq.clone()) for _ in range(layers - 1)]
+    for i in range(2 * layers):
+        M.mla_query_proj(dims, h, *mats[i % layers], c_q, q, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(iters):
+        M.mla_query_proj(dims, h, *mats[i % layers], c_q, q, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    b2b_us = e0.elapsed_time(e1) * 1000.0 / iters
+    del mats
     return {"time_us": us, "bytes_per_launch": nbytes, "launches": 2 * iters, "tokens": w.tokens,
+            "layers_us": b2b_us, "layers": layers,
+            "layers_bytes": layers * (w_dq.numel() + w_uq.numel()) * 2,
             "shape": f"c_Q[{w.tokens}, {r}] = h[{w.tokens}, {w.d_model}] . W_DQ^T; "
                      f"q[{w.tokens}, {w.n_heads}, {w.qk_nope + w.d_rope}] = c_Q . W_UQ^T"}
 
@@ -751,7 +773,12 @@ def main():
             "kernel": "token_linear_kernel x 2 (mla_query_proj), timed alone after the step, not part of it",
             "shape": qp["shape"], "bound": "hbm", "achieved": qp_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": qp_gbs / peaks["hbm_gbs"], "time_us": qp["time_us"], "bytes_per_call": qp["bytes_per_launch"],
-            "launches_timed": qp["launches"], "l2": "256 MB buffer rewritten before each call"}
+            "launches_timed": qp["launches"], "l2": "256 MB buffer rewritten before each call",
+            "layers_back_to_back": {
+                "time_us": qp["layers_us"],
+                "frac": qp["bytes_per_launch"] / (qp["layers_us"] * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                "l2": f"{qp['layers']} layers' W_DQ and W_UQ ({qp['layers_bytes'] / 1e6:.0f} MB) in turn, "
+                      "back to back, no flush"}}
         pf = r["prefill"]
         pf_tfs = pf["flops"] / (pf["time_us"] * 1e-6) / 1e12
         line["next_rows"]["prefill"] = {
