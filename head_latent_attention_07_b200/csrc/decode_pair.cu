@@ -286,6 +286,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     const uint32_t kfull0 = mapa(smem_u32(&bar->kfull[0]), 0);
     const uint32_t qfull0 = mapa(smem_u32(&bar->q_full), 0);
     const int oob_row = a.num_pages * 64;   // a box starting here lies outside the pool: zero fill
+    const uint64_t stream_policy = l2_policy_evict_first();   // pages are read once per call
     StepCursor cur(plan, a.batch, w);
     Step st;
     int t = 0;
@@ -314,14 +315,14 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         mbar_arrive_expect_tx_cluster(kfull0 + 8 * u, kBufBytes);
         for (int k = 0; k < 5; ++k) {             // blocks 0, 1, 4, 5, 8
           const int blk = k == 4 ? 8 : (k & 1) + 4 * (k >> 1);
-          tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+          tma_load_2d_pair_hint(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u, stream_policy);
         }
       }
       if (t >= 2 && !wwait(&bar->buf_free[u], ((t >> 1) - 1) & 1)) break;
       if (lane == 0)
         for (int k = 0; k < 4; ++k) {             // blocks 2, 3, 6, 7
           const int blk = 2 + (k & 1) + 4 * (k >> 1);
-          tma_load_2d_pair(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u);
+          tma_load_2d_pair_hint(dst + blk * kBlockBytes, &tp, 64 * blk, y, kfull0 + 8 * u, stream_policy);
         }
       ++t;
     }
@@ -337,6 +338,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     // hands the step on.
     const char* pool = reinterpret_cast<const char*>(a.pool);
     const uint32_t vfull0 = mapa(smem_u32(&bar->vfull[0]), 0);
+    const uint64_t stream_policy = l2_policy_evict_first();
     StepCursor cur(plan, a.batch, w);
     Step st;
     int t = 0;
@@ -353,8 +355,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
           mbar_arrive_expect_tx_cluster(vfull0 + 8 * u, 4 * kBlockBytes);
           for (int je = 0; je < 4; ++je) {
             const int j = je >> 1, e = je & 1;
-            tma_load_2d_pair(buf + (4 * j + 2 * pp + e) * kBlockBytes, &tp, 256 * j + 128 * (int)c + 64 * e,
-                             f.id_p * 64, vfull0 + 8 * u);
+            tma_load_2d_pair_hint(buf + (4 * j + 2 * pp + e) * kBlockBytes, &tp, 256 * j + 128 * (int)c + 64 * e,
+                                  f.id_p * 64, vfull0 + 8 * u, stream_policy);
           }
         }
         __syncwarp();
@@ -390,6 +392,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
   } else if (warp == 3) {
     // ------------------------------------------------------------ hand a partial step's value operand on
     const uint32_t vfull0 = mapa(smem_u32(&bar->vfull[0]), 0);
+    const uint64_t stream_policy = l2_policy_evict_first();
     StepCursor cur(plan, a.batch, w);
     Step st;
     int t = 0;
