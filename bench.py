@@ -153,6 +153,13 @@ def job_throughput(world: int, tokens_per_rank: int, steps: int, ms: float) -> f
     return world * tokens_per_rank * steps / (ms / 1000.0)
 
 
+def layer_copies(nbytes_per_layer: int) -> int:
+    """How many copies of one layer's weights a back-to-back loop cycles through
+    so that a copy is evicted from L2 before its next use: their total exceeds
+    twice the L2, with at least two copies."""
+    return max(2, -(-2 * L2_BYTES // nbytes_per_layer) + 1)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -565,7 +572,7 @@ def measure_query_proj(M, w: W.Workload, dims, dev, stream, seed: int, iters: in
     nbytes = (w_dq.numel() + w_uq.numel() + h.numel() + 2 * c_q.numel() + q.numel()) * 2
     # as a model's layers run it: back-to-back calls, each with another layer's
     # weights (copies whose total exceeds twice the L2), no flush in between
-    layers = max(2, -(-2 * L2_BYTES // ((w_dq.numel() + w_uq.numel()) * 2)) + 1)
+    layers = layer_copies((w_dq.numel() + w_uq.numel()) * 2)
     mats = [(w_dq, w_uq)] + [(w_dq.clone(), w_uq.clone()) for _ in range(layers - 1)]
     for i in range(2 * layers):
         M.mla_query_proj(dims, h, *mats[i % layers], c_q, q, stream=stream)

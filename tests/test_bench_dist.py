@@ -70,3 +70,13 @@ def test_reference_arm_non_zero_rank_exits_quietly():
                         "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_layer_copies_exceed_twice_l2():
+    # the query path's weights at the V3 shape (W_DQ 22.0 MB + W_UQ 75.5 MB)
+    per = (1536 * 7168 + 128 * 192 * 1536) * 2
+    n = bench.layer_copies(per)
+    assert n == 4 and n * per > 2 * bench.L2_BYTES and (n - 1) * per <= 2 * bench.L2_BYTES + per
+    # small layers need many copies, huge ones still two
+    assert bench.layer_copies(1 << 20) * (1 << 20) > 2 * bench.L2_BYTES
+    assert bench.layer_copies(10 * bench.L2_BYTES) == 2
