@@ -107,7 +107,7 @@ def algorithmic_counts(w: W.Workload, lens: np.ndarray) -> dict:
 
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_pair_kernel_v3.md")
 KERNEL_SOURCES = ["decode_pair.cu", "decode_combine.cu", "plan.cuh", "sm100.cuh", "common.cuh", "mma_frag.cuh",
-                  "decode.h"]
+                  "decode.h", "tma_map.cu", "api.cu"]   # the kernels, their tensor maps and launch shapes
 
 
 def kernel_sources_sha256() -> str:
